@@ -1,0 +1,233 @@
+/*
+ * dp.h — C ABI of the DualParal window-step library for NVIDIA B200 (sm_100a).
+ *
+ * The method ("Minute-Long Videos with Dual Parallelisms", arXiv 2505.21070, abstract;
+ * pith.science review of the same paper, Sections 3.1-3.2 and Figure 1) denoises a FIFO
+ * queue of temporal blocks of latent frames, each block at its own (staggered) noise
+ * level, in one DiT forward per step.  Every block's tokens attend to the window's own K/V
+ * plus the cached K/V features of the block that last left the queue; each step pushes a
+ * noisy block at the tail and pops a clean block at the head.  This library computes, on
+ * one GPU, the per-step hot path of that scheme:
+ *
+ *   A0  per-block adaLN lookup (host)         dp_blocks_from_table, dp_queue_blocks
+ *   A1  K/V modulation prepass                dp_adaln_modulate
+ *   A2  window attention over [cache ; window] with the Q modulation fused into its
+ *       prologue and the gate (+ residual) into its epilogue   dp_window_attention
+ *   A3  queue and cache advance               dp_kvcache_advance, dp_queue_push/pop
+ *   A4  the whole step A1 -> A2 -> A3         dp_window_step
+ *
+ * Conventions (all entry points):
+ *  - Token tensors are row-major [rows][hidden], hidden = n_heads * head_dim, channel
+ *    c = h * head_dim + d.  Window rows are ordered head block (cleanest, smallest
+ *    timestep) first.
+ *  - Element type is given by dp_dtype: DP_BF16 (bfloat16) or DP_F32 (float).  adaLN
+ *    vectors are always float.
+ *  - Ownership: the caller owns every device buffer; the library allocates no device
+ *    memory on any call.  Descriptor structs are host-side plain data; the library
+ *    updates their counters deterministically.
+ *  - Asynchrony: work is enqueued on the given stream (a cudaStream_t; NULL = the legacy
+ *    default stream) of the current device (see dp_set_device).  Argument errors are
+ *    returned synchronously before anything is enqueued and leave descriptors unchanged.
+ *  - Alignment: every device pointer must be 16-byte aligned and hidden * element size a
+ *    multiple of 16 bytes.
+ *  - Errors: launch failures return DP_ERR_CUDA (dp_last_error_detail() gives the CUDA
+ *    message).  Bounded device-side waits that give up record DP_ERR_TIMEOUT in a device
+ *    status word read by dp_device_status(); the kernel then returns without hanging.
+ */
+#ifndef DP_H
+#define DP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DP_MAX_BLOCKS 16   /* blocks in one window */
+#define DP_MAX_SLOTS 16    /* slots of the latent queue and of the cache ring */
+
+typedef enum {
+  DP_OK = 0,
+  DP_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, inconsistent sizes or offsets */
+  DP_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. bf16 head_dim not 64/128) */
+  DP_ERR_CUDA = -3,         /* a CUDA call or kernel launch failed */
+  DP_ERR_CAPACITY = -4,     /* a block does not fit its cache slot / queue slot / queue */
+  DP_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (see dp_device_status) */
+  DP_ERR_EMPTY = -6         /* pop from an empty queue */
+} dp_status;
+
+typedef enum { DP_F32 = 0, DP_BF16 = 1 } dp_dtype;
+
+/* dp_window_attention flags */
+#define DP_MOD_Q 1u     /* prologue: q' = q * (1 + scale_b) + shift_b, b = block of the row */
+#define DP_GATE_OUT 2u  /* epilogue: out = gate_b * o (+ residual) */
+
+/* dp_window_step flags */
+#define DP_STEP_POP 1u  /* after attention, the head block exits: its K'/V' rows become the
+                           cache (and the queue, if given, pops its head) */
+
+/*
+ * Window block table (host plain data, passed by pointer, copied into kernel arguments).
+ * Block b owns window rows [row_offset[b], row_offset[b+1]); row_offset[0] = 0, offsets
+ * non-decreasing, row_offset[n_blocks] = the window's row count.  mod[b] is a DEVICE
+ * pointer to 3 * hidden floats: shift[hidden], scale[hidden], gate[hidden] — block b's
+ * adaLN vectors for its own timestep (the review's Section 3.1: neighbouring blocks sit
+ * at neighbouring noise levels; the DiT conditions each block on its own timestep).
+ */
+typedef struct {
+  int32_t n_blocks;
+  int32_t hidden;
+  int32_t row_offset[DP_MAX_BLOCKS + 1];
+  const float* mod[DP_MAX_BLOCKS];
+} dp_blocks;
+
+/*
+ * Feature cache (the review's Section 3.2: the self-attention K/V features of the block
+ * that just left, reused as context, one denoising step stale).  A ring of n_slots slots,
+ * each [capacity][hidden] in k and in v (DEVICE, caller-owned, [n_slots][capacity][hidden]).
+ * An advance writes slot (n_advances mod n_slots); attention reads the most recently
+ * written slot (slot 0 before the first advance, whose contents the caller may preset
+ * together with len[0]).
+ */
+typedef struct {
+  void* k;
+  void* v;
+  int64_t capacity;
+  int32_t hidden;
+  int32_t n_slots;
+  int64_t len[DP_MAX_SLOTS];
+  int64_t n_advances;
+  dp_dtype dtype;
+} dp_kvcache;
+
+/*
+ * Latent block queue (the review's key machinery: a FIFO of blocks with noise levels
+ * decreasing from tail to head).  latent is DEVICE memory [2 * n_slots][slot_rows][hidden],
+ * a mirrored ring: a block pushed to physical slot p is written to slots p and p + n_slots,
+ * so the live window, slots [head, head + count), is always one contiguous range.
+ * rows[i] and evals[i] describe the block at logical position i (0 = head).  Only the
+ * tail block may hold fewer than slot_rows rows (a ragged final block); no push may
+ * follow it.
+ */
+typedef struct {
+  void* latent;
+  int64_t slot_rows;
+  int32_t hidden;
+  int32_t n_slots;
+  int32_t head;
+  int32_t count;
+  int32_t rows[DP_MAX_SLOTS];
+  int32_t evals[DP_MAX_SLOTS];
+  int64_t n_pushed;
+  int64_t n_popped;
+  dp_dtype dtype;
+} dp_queue;
+
+/* ---------------------------------------------------------------- A0: host lookups */
+
+/* Fill *out for n_blocks blocks: rows block_rows[b] (host), adaLN row table[timesteps[b]]
+ * (the table is DEVICE memory [table_rows][3][hidden] float, standing in for the DiT's
+ * timestep MLP).  INVALID_ARG on a timestep outside [0, table_rows) or n_blocks outside
+ * [1, DP_MAX_BLOCKS]. */
+dp_status dp_blocks_from_table(dp_blocks* out, const float* table, int32_t table_rows,
+                               int32_t hidden, const int32_t* timesteps,
+                               const int32_t* block_rows, int32_t n_blocks);
+
+/* Block table of the queue's live window: block i gets rows[i] and adaLN row
+ * table[tau[evals[i]]] (tau: host array of n_tau timesteps, noisiest first).  *window
+ * receives the DEVICE address of the head block's first row (q = k = v of the window),
+ * *n_win the window's row count.  EMPTY if no block is live; INVALID_ARG if a block has
+ * already had n_tau evaluations. */
+dp_status dp_queue_blocks(const dp_queue* q, const float* table, int32_t table_rows,
+                          const int32_t* tau, int32_t n_tau, dp_blocks* out,
+                          const void** window, int64_t* n_win);
+
+/* ---------------------------------------------------------------- A1: modulation */
+
+/* y[i, c] = x[i, c] * (1 + scale_b[c]) + shift_b[c] for every row i of block b, in fp32
+ * (one fused multiply-add, 1 + scale rounded to float), rounded to the element type.
+ * x, y: DEVICE [n_rows][hidden]; y may equal x (in place), no other overlap.
+ * n_rows must equal blk->row_offset[blk->n_blocks]. */
+dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blocks* blk,
+                            dp_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------- A2: attention */
+
+/* Window attention (the abstract's feature cache reused as context; the review's
+ * Section 3.2 self-attention over the cached K/V of the neighbouring block):
+ *   q'_i  = DP_MOD_Q ? q_i * (1 + scale_b) + shift_b : q_i          (b = block of row i)
+ *   o_i,h = sum_j softmax_j(q'_i,h . K_j,h * softmax_scale) V_j,h,
+ *           j over cache rows [0, cache_len) then window rows [0, n_win)
+ *   out_i = (DP_GATE_OUT ? gate_b * o_i : o_i) + (residual ? residual_i : 0)
+ * q, k, v, residual, out: DEVICE [n_win][hidden]; k and v enter as given (the window's
+ * modulated features).  cache_k, cache_v: DEVICE, at least cache_len rows.  residual may
+ * be NULL.  out must not overlap any input.  softmax_scale <= 0 selects 1/sqrt(head_dim).
+ * bf16: head_dim 64 or 128 (tensor cores, fp32 accumulation and softmax); f32: head_dim
+ * a multiple of 4 up to 128 (CUDA cores, full fp32).  UNSUPPORTED otherwise. */
+dp_status dp_window_attention(const void* q, const void* k, const void* v, int64_t n_win,
+                              const void* cache_k, const void* cache_v, int64_t cache_len,
+                              const void* residual, void* out, int32_t n_heads,
+                              int32_t head_dim, float softmax_scale, const dp_blocks* blk,
+                              uint32_t flags, dp_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------- A3: advance */
+
+/* The exiting head block's features become the cache: rows [0, n_exit) of k_exit and
+ * v_exit (DEVICE [n_exit][hidden]) are copied into slot (n_advances mod n_slots);
+ * len[slot] = n_exit; n_advances += 1.  A byte copy (bit-exact).  CAPACITY if n_exit >
+ * capacity.  n_exit = 0 empties the slot. */
+dp_status dp_kvcache_advance(dp_kvcache* c, const void* k_exit, const void* v_exit,
+                             int64_t n_exit, void* stream);
+
+/* Push a fresh noise block (DEVICE [rows][hidden]) at the queue's tail (byte copy into the
+ * mirrored ring); the new block has evals = 0.  CAPACITY if the queue is full or rows >
+ * slot_rows; INVALID_ARG if the current tail is a short (final) block. */
+dp_status dp_queue_push(dp_queue* q, const void* noise, int64_t rows, void* stream);
+
+/* Pop the head block (metadata only: the slot becomes free).  EMPTY if no block. */
+dp_status dp_queue_pop(dp_queue* q);
+
+/* ---------------------------------------------------------------- A4: window step */
+
+/* One window step:
+ *   1. k' = modulate(k), v' = modulate(v) into kv_work (DEVICE scratch, caller-allocated,
+ *      2 * n_win * hidden elements: k' then v');
+ *   2. out = dp_window_attention(q, k', v', cache, DP_MOD_Q | DP_GATE_OUT, residual);
+ *   3. queue (if given): every live block's evals += 1;
+ *   4. if flags & DP_STEP_POP: the head block (rows [0, row_offset[1])) exits — its k'/v'
+ *      rows are written into the cache ring (dp_kvcache_advance), and the queue (if
+ *      given) pops its head;
+ *   5. if push_noise: it is pushed at the queue's tail (dp_queue_push; needs queue).
+ * Steps 4 and 5 run as one copy kernel after the attention on the same stream.  All
+ * argument checks (including capacities) happen before anything is enqueued.  q, k and v
+ * may alias one another (the queue's window); out and kv_work overlap nothing. */
+dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_win,
+                         const dp_blocks* blk, dp_kvcache* cache, void* kv_work,
+                         const void* residual, void* out, int32_t n_heads, int32_t head_dim,
+                         uint32_t flags, dp_queue* queue, const void* push_noise,
+                         int64_t push_rows, dp_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Make device `ordinal` current for this thread's later calls. */
+dp_status dp_set_device(int32_t ordinal);
+
+/* Synchronize `stream`, then read and clear the device status word of the current device:
+ * DP_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call, else DP_OK
+ * (or DP_ERR_CUDA if the synchronize failed). */
+dp_status dp_device_status(void* stream);
+
+/* Static text for a status code. */
+const char* dp_status_string(dp_status s);
+
+/* Detail of the most recent failure on this thread (CUDA error text, failed check). */
+const char* dp_last_error_detail(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t dp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DP_H */

@@ -1,0 +1,301 @@
+"""Python binding of the DualParal window-step library (libdp_b200.so, sm_100a).
+
+Argument marshalling only: every step of the window step runs in the library's CUDA
+kernels, and there is no fallback.  Importing fails loudly when the library has not been
+built (``python -m long_video_diffusion_b200._build``).  PyTorch supplies device memory,
+streams and the current device; tensors are passed as raw pointers.
+
+The calls mirror include/dp.h:
+  blocks_from_table, queue_blocks   A0  per-block adaLN lookup (host)
+  adaln_modulate                    A1  modulation prepass
+  window_attention                  A2  attention over [cache ; window], fused Q prologue
+                                        and gate (+ residual) epilogue
+  kvcache_advance, queue_push/pop   A3  queue and cache advance
+  window_step                       A4  the whole step
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdp_b200.so")
+
+MAX_BLOCKS = 16
+MAX_SLOTS = 16
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_CAPACITY, ERR_TIMEOUT, ERR_EMPTY = 0, -1, -2, -3, -4, -5, -6
+F32, BF16 = 0, 1
+MOD_Q, GATE_OUT = 1, 2
+STEP_POP = 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_video_diffusion_b200._build` "
+                      "(nvcc, sm_100a). There is no non-CUDA implementation.")
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class DpBlocks(ctypes.Structure):
+    _fields_ = [("n_blocks", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("row_offset", ctypes.c_int32 * (MAX_BLOCKS + 1)),
+                ("mod", ctypes.c_void_p * MAX_BLOCKS)]
+
+    @property
+    def offsets(self):
+        return [self.row_offset[i] for i in range(self.n_blocks + 1)]
+
+
+class DpKvcache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("hidden", ctypes.c_int32), ("n_slots", ctypes.c_int32),
+                ("len", ctypes.c_int64 * MAX_SLOTS), ("n_advances", ctypes.c_int64),
+                ("dtype", ctypes.c_int32)]
+
+
+class DpQueue(ctypes.Structure):
+    _fields_ = [("latent", ctypes.c_void_p), ("slot_rows", ctypes.c_int64), ("hidden", ctypes.c_int32),
+                ("n_slots", ctypes.c_int32), ("head", ctypes.c_int32), ("count", ctypes.c_int32),
+                ("rows", ctypes.c_int32 * MAX_SLOTS), ("evals", ctypes.c_int32 * MAX_SLOTS),
+                ("n_pushed", ctypes.c_int64), ("n_popped", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I32, _I64, _U32, _F = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
+_SIGS = {
+    "dp_blocks_from_table": [ctypes.POINTER(DpBlocks), _P, _I32, _I32, ctypes.POINTER(_I32),
+                             ctypes.POINTER(_I32), _I32],
+    "dp_queue_blocks": [ctypes.POINTER(DpQueue), _P, _I32, ctypes.POINTER(_I32), _I32,
+                        ctypes.POINTER(DpBlocks), ctypes.POINTER(_P), ctypes.POINTER(_I64)],
+    "dp_adaln_modulate": [_P, _P, _I64, ctypes.POINTER(DpBlocks), _I32, _P],
+    "dp_window_attention": [_P, _P, _P, _I64, _P, _P, _I64, _P, _P, _I32, _I32, _F,
+                            ctypes.POINTER(DpBlocks), _U32, _I32, _P],
+    "dp_kvcache_advance": [ctypes.POINTER(DpKvcache), _P, _P, _I64, _P],
+    "dp_queue_push": [ctypes.POINTER(DpQueue), _P, _I64, _P],
+    "dp_queue_pop": [ctypes.POINTER(DpQueue)],
+    "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
+                       _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
+    "dp_set_device": [_I32],
+    "dp_device_status": [_P],
+    "dp_status_string": [_I32],
+    "dp_last_error_detail": [],
+    "dp_version": [],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int32
+_lib.dp_status_string.restype = ctypes.c_char_p
+_lib.dp_last_error_detail.restype = ctypes.c_char_p
+
+EXPORTS = sorted(_SIGS)
+
+
+class DpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        detail = _lib.dp_last_error_detail().decode(errors="replace")
+        name = _lib.dp_status_string(status).decode()
+        super().__init__(f"{where}: {name} ({detail})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise DpError(status, where)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor, stream=None):
+    dev = t.device.index if t.device.index is not None else torch.cuda.current_device()
+    _check(_lib.dp_set_device(dev), "dp_set_device")
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def version() -> int:
+    return _lib.dp_version()
+
+
+# ------------------------------------------------------------------------- A0
+
+def blocks_from_table(table: torch.Tensor, timesteps: Sequence[int], block_rows: Sequence[int]) -> DpBlocks:
+    """Block table whose block b uses rows block_rows[b] and adaLN row table[timesteps[b]]."""
+    if table.dtype != torch.float32 or table.dim() != 3 or table.shape[1] != 3:
+        raise ValueError("table must be float32 [T, 3, hidden]")
+    n = len(timesteps)
+    if len(block_rows) != n:
+        raise ValueError("timesteps and block_rows differ in length")
+    out = DpBlocks()
+    ts = (ctypes.c_int32 * max(n, 1))(*timesteps)
+    rows = (ctypes.c_int32 * max(n, 1))(*block_rows)
+    _check(_lib.dp_blocks_from_table(ctypes.byref(out), _ptr(table), table.shape[0], table.shape[2], ts, rows, n),
+           "dp_blocks_from_table")
+    out._table = table  # keep the table alive while the block table is in use
+    return out
+
+
+# ------------------------------------------------------------------------- state
+
+class KVCache:
+    """The feature-cache ring (device buffers [n_slots, capacity, hidden] owned here)."""
+
+    def __init__(self, capacity: int, hidden: int, dtype=torch.bfloat16, n_slots: int = 1,
+                 device="cuda", k: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None,
+                 length: int = 0):
+        self.k = torch.zeros(n_slots, capacity, hidden, dtype=dtype, device=device) if k is None else k
+        self.v = torch.zeros(n_slots, capacity, hidden, dtype=dtype, device=device) if v is None else v
+        if self.k.shape != (n_slots, capacity, hidden) or self.v.shape != self.k.shape:
+            raise ValueError("cache buffers must be [n_slots, capacity, hidden]")
+        self.desc = DpKvcache()
+        self.desc.k = self.k.data_ptr()
+        self.desc.v = self.v.data_ptr()
+        self.desc.capacity = capacity
+        self.desc.hidden = hidden
+        self.desc.n_slots = n_slots
+        self.desc.len[0] = length
+        self.desc.n_advances = 0
+        self.desc.dtype = _dtype(self.k)
+
+    @property
+    def n_advances(self) -> int:
+        return self.desc.n_advances
+
+    def read_slot(self) -> int:
+        d = self.desc
+        return (d.n_advances - 1) % d.n_slots if d.n_advances > 0 else 0
+
+    @property
+    def length(self) -> int:
+        return self.desc.len[self.read_slot()]
+
+
+class Queue:
+    """The latent block queue: a mirrored ring [2 * n_slots, slot_rows, hidden] owned here."""
+
+    def __init__(self, n_slots: int, slot_rows: int, hidden: int, dtype=torch.bfloat16, device="cuda"):
+        self.latent = torch.zeros(2 * n_slots, slot_rows, hidden, dtype=dtype, device=device)
+        self.desc = DpQueue()
+        self.desc.latent = self.latent.data_ptr()
+        self.desc.slot_rows = slot_rows
+        self.desc.hidden = hidden
+        self.desc.n_slots = n_slots
+        self.desc.head = 0
+        self.desc.count = 0
+        self.desc.dtype = _dtype(self.latent)
+
+    @property
+    def count(self) -> int:
+        return self.desc.count
+
+    @property
+    def head(self) -> int:
+        return self.desc.head
+
+    def rows(self):
+        return [self.desc.rows[i] for i in range(self.desc.count)]
+
+    def evals(self):
+        return [self.desc.evals[i] for i in range(self.desc.count)]
+
+    def window_rows(self) -> int:
+        return sum(self.rows())
+
+    def window(self) -> torch.Tensor:
+        """View of the live window (head block first) inside the mirrored ring."""
+        flat = self.latent.view(-1, self.desc.hidden)
+        start = self.desc.head * self.desc.slot_rows
+        return flat[start:start + self.window_rows()]
+
+
+def queue_blocks(queue: Queue, table: torch.Tensor, tau: Sequence[int]):
+    """(block table, window pointer, n_win) of the queue's live window."""
+    out = DpBlocks()
+    tarr = (ctypes.c_int32 * len(tau))(*tau)
+    win = ctypes.c_void_p()
+    n = ctypes.c_int64()
+    _check(_lib.dp_queue_blocks(ctypes.byref(queue.desc), _ptr(table), table.shape[0], tarr, len(tau),
+                                ctypes.byref(out), ctypes.byref(win), ctypes.byref(n)), "dp_queue_blocks")
+    out._table = table
+    return out, win.value, n.value
+
+
+# ------------------------------------------------------------------------- A1..A4
+
+def adaln_modulate(x: torch.Tensor, y: torch.Tensor, blocks: DpBlocks, stream=None) -> None:
+    _check(_lib.dp_adaln_modulate(_ptr(x), _ptr(y), x.shape[0], ctypes.byref(blocks), _dtype(x),
+                                  _stream(x, stream)), "dp_adaln_modulate")
+
+
+def window_attention(q, k, v, cache_k, cache_v, cache_len: int, out, n_heads: int, head_dim: int,
+                     blocks: DpBlocks, flags: int = MOD_Q | GATE_OUT, residual=None,
+                     softmax_scale: float = 0.0, stream=None) -> None:
+    _check(_lib.dp_window_attention(_ptr(q), _ptr(k), _ptr(v), q.shape[0], _ptr(cache_k), _ptr(cache_v),
+                                    int(cache_len), _ptr(residual), _ptr(out), n_heads, head_dim,
+                                    float(softmax_scale), ctypes.byref(blocks), flags, _dtype(q),
+                                    _stream(q, stream)), "dp_window_attention")
+
+
+def kvcache_advance(cache: KVCache, k_exit: torch.Tensor, v_exit: torch.Tensor, n_exit: int, stream=None) -> None:
+    _check(_lib.dp_kvcache_advance(ctypes.byref(cache.desc), _ptr(k_exit), _ptr(v_exit), int(n_exit),
+                                   _stream(cache.k, stream)), "dp_kvcache_advance")
+
+
+def queue_push(queue: Queue, noise: torch.Tensor, rows: Optional[int] = None, stream=None) -> None:
+    r = noise.shape[0] if rows is None else rows
+    _check(_lib.dp_queue_push(ctypes.byref(queue.desc), _ptr(noise), int(r), _stream(queue.latent, stream)),
+           "dp_queue_push")
+
+
+def queue_pop(queue: Queue) -> None:
+    _check(_lib.dp_queue_pop(ctypes.byref(queue.desc)), "dp_queue_pop")
+
+
+def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads: int, head_dim: int,
+                pop: bool = False, queue: Optional[Queue] = None, push_noise=None, push_rows=None,
+                residual=None, stream=None, n_win: Optional[int] = None) -> None:
+    """One window step (see dp_window_step).  q, k, v are tensors or raw device addresses
+    (n_win then required), e.g. the queue's live window."""
+    if isinstance(q, torch.Tensor):
+        ref = q
+        n = q.shape[0]
+        qp, kp, vp = _ptr(q), _ptr(k), _ptr(v)
+    else:
+        ref = out
+        n = int(n_win)
+        qp, kp, vp = ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v)
+    rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
+    _check(_lib.dp_window_step(qp, kp, vp, n, ctypes.byref(blocks), ctypes.byref(cache.desc), _ptr(kv_work),
+                               _ptr(residual), _ptr(out), n_heads, head_dim, STEP_POP if pop else 0,
+                               ctypes.byref(queue.desc) if queue is not None else None, _ptr(push_noise),
+                               int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
+
+
+def device_status(stream=None) -> int:
+    """Synchronize and read/clear the device status word; raises DpError on a timeout."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    st = _lib.dp_device_status(ctypes.c_void_p(s.cuda_stream))
+    _check(st, "dp_device_status")
+    return st
+
+
+def loaded_library_path() -> str:
+    return LIB_PATH

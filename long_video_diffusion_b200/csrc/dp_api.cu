@@ -1,0 +1,454 @@
+// C ABI of the window-step library: argument checks, descriptor bookkeeping, launches.
+// The operations and their sources are documented in include/dp.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "dp.h"
+#include "dp_internal.h"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+dp_status fail(dp_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+dp_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(DP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(dp_dtype dt) { return dt == DP_BF16 ? 2 : 4; }
+
+bool dtype_ok(dp_dtype dt) { return dt == DP_BF16 || dt == DP_F32; }
+
+// Row pitch must be a whole number of 16-byte vectors.
+bool hidden_ok(int32_t hidden, dp_dtype dt) {
+  return hidden > 0 && (static_cast<int64_t>(hidden) * elem_bytes(dt)) % 16 == 0;
+}
+
+dp_status check_blocks(const dp_blocks* blk, int64_t n_rows, int32_t hidden) {
+  if (!blk) return fail(DP_ERR_INVALID_ARG, "block table is NULL");
+  if (blk->n_blocks < 1 || blk->n_blocks > DP_MAX_BLOCKS)
+    return fail(DP_ERR_INVALID_ARG, "n_blocks %d outside [1, %d]", blk->n_blocks, DP_MAX_BLOCKS);
+  if (blk->hidden != hidden) return fail(DP_ERR_INVALID_ARG, "block table hidden %d != %d", blk->hidden, hidden);
+  if (blk->row_offset[0] != 0) return fail(DP_ERR_INVALID_ARG, "row_offset[0] must be 0");
+  for (int b = 0; b < blk->n_blocks; ++b) {
+    if (blk->row_offset[b + 1] < blk->row_offset[b]) return fail(DP_ERR_INVALID_ARG, "row_offset decreases at %d", b);
+    if (!blk->mod[b] || !aligned16(blk->mod[b])) return fail(DP_ERR_INVALID_ARG, "mod[%d] NULL or misaligned", b);
+  }
+  if (blk->row_offset[blk->n_blocks] != n_rows)
+    return fail(DP_ERR_INVALID_ARG, "row_offset[n_blocks] = %d != rows %lld", blk->row_offset[blk->n_blocks],
+                static_cast<long long>(n_rows));
+  return DP_OK;
+}
+
+dp::BlockTable to_table(const dp_blocks* blk) {
+  dp::BlockTable t;
+  memset(&t, 0, sizeof(t));
+  t.n_blocks = blk->n_blocks;
+  for (int b = 0; b <= blk->n_blocks; ++b) t.row_offset[b] = blk->row_offset[b];
+  for (int b = blk->n_blocks + 1; b <= DP_MAX_BLOCKS; ++b) t.row_offset[b] = blk->row_offset[blk->n_blocks];
+  for (int b = 0; b < blk->n_blocks; ++b) t.mod[b] = blk->mod[b];
+  for (int b = blk->n_blocks; b < DP_MAX_BLOCKS; ++b) t.mod[b] = blk->mod[0];
+  return t;
+}
+
+constexpr int kMaxDevices = 64;
+uint32_t* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+}  // namespace
+
+// The device status word bounded waits write to (one per device that loads the library).
+__device__ uint32_t dp_status_word;
+
+namespace {
+
+dp_status status_ptr(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DP_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, dp_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    g_status_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return DP_OK;
+}
+
+int64_t cache_read_slot(const dp_kvcache* c) {
+  return c->n_advances > 0 ? (c->n_advances - 1) % c->n_slots : 0;
+}
+
+dp_status check_cache(const dp_kvcache* c, int32_t hidden, dp_dtype dt) {
+  if (!c) return fail(DP_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->k || !c->v || !aligned16(c->k) || !aligned16(c->v))
+    return fail(DP_ERR_INVALID_ARG, "cache k/v NULL or misaligned");
+  if (c->hidden != hidden || c->dtype != dt) return fail(DP_ERR_INVALID_ARG, "cache hidden/dtype mismatch");
+  if (c->n_slots < 1 || c->n_slots > DP_MAX_SLOTS) return fail(DP_ERR_INVALID_ARG, "cache n_slots %d", c->n_slots);
+  if (c->capacity < 0 || c->n_advances < 0) return fail(DP_ERR_INVALID_ARG, "cache capacity/n_advances negative");
+  for (int s = 0; s < c->n_slots; ++s)
+    if (c->len[s] < 0 || c->len[s] > c->capacity)
+      return fail(DP_ERR_CAPACITY, "cache len[%d] = %lld outside [0, capacity]", s, static_cast<long long>(c->len[s]));
+  return DP_OK;
+}
+
+dp_status check_queue(const dp_queue* q, int32_t hidden, dp_dtype dt) {
+  if (!q->latent || !aligned16(q->latent)) return fail(DP_ERR_INVALID_ARG, "queue latent NULL or misaligned");
+  if (q->hidden != hidden || q->dtype != dt) return fail(DP_ERR_INVALID_ARG, "queue hidden/dtype mismatch");
+  if (q->n_slots < 1 || q->n_slots > DP_MAX_SLOTS) return fail(DP_ERR_INVALID_ARG, "queue n_slots %d", q->n_slots);
+  if (q->count < 0 || q->count > q->n_slots || q->head < 0 || q->head >= q->n_slots || q->slot_rows <= 0)
+    return fail(DP_ERR_INVALID_ARG, "queue head/count/slot_rows inconsistent");
+  return DP_OK;
+}
+
+// Physical slot p of the mirrored ring: copies land at slots p and p + n_slots.
+char* queue_slot(const dp_queue* q, int32_t p) {
+  const int64_t pitch = q->slot_rows * q->hidden * elem_bytes(q->dtype);
+  return static_cast<char*>(q->latent) + static_cast<int64_t>(p) * pitch;
+}
+
+dp_status check_push(const dp_queue* q, int32_t count_after_pop, const void* noise, int64_t rows) {
+  if (!noise || !aligned16(noise)) return fail(DP_ERR_INVALID_ARG, "push noise NULL or misaligned");
+  if (rows <= 0) return fail(DP_ERR_INVALID_ARG, "push rows %lld", static_cast<long long>(rows));
+  if (rows > q->slot_rows) return fail(DP_ERR_CAPACITY, "push rows %lld > slot_rows", static_cast<long long>(rows));
+  if (count_after_pop >= q->n_slots) return fail(DP_ERR_CAPACITY, "queue full (%d blocks)", q->n_slots);
+  if (count_after_pop > 0) {
+    // the tail is the block at logical position count_after_pop - 1 (after any pop)
+    const int shift = q->count - count_after_pop;  // 1 if the head was popped
+    const int32_t tail_rows = q->rows[count_after_pop - 1 + shift];
+    if (tail_rows < q->slot_rows) return fail(DP_ERR_INVALID_ARG, "no push may follow a short final block");
+  }
+  return DP_OK;
+}
+
+void apply_pop(dp_queue* q) {
+  for (int i = 1; i < q->count; ++i) {
+    q->rows[i - 1] = q->rows[i];
+    q->evals[i - 1] = q->evals[i];
+  }
+  q->count -= 1;
+  q->rows[q->count] = 0;
+  q->evals[q->count] = 0;
+  q->head = (q->head + 1) % q->n_slots;
+  q->n_popped += 1;
+}
+
+int32_t apply_push(dp_queue* q, int64_t rows) {
+  const int32_t p = (q->head + q->count) % q->n_slots;
+  q->rows[q->count] = static_cast<int32_t>(rows);
+  q->evals[q->count] = 0;
+  q->count += 1;
+  q->n_pushed += 1;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dp_version(void) { return 100; }
+
+const char* dp_status_string(dp_status s) {
+  switch (s) {
+    case DP_OK: return "DP_OK";
+    case DP_ERR_INVALID_ARG: return "DP_ERR_INVALID_ARG";
+    case DP_ERR_UNSUPPORTED: return "DP_ERR_UNSUPPORTED";
+    case DP_ERR_CUDA: return "DP_ERR_CUDA";
+    case DP_ERR_CAPACITY: return "DP_ERR_CAPACITY";
+    case DP_ERR_TIMEOUT: return "DP_ERR_TIMEOUT";
+    case DP_ERR_EMPTY: return "DP_ERR_EMPTY";
+  }
+  return "DP_ERR_UNKNOWN";
+}
+
+const char* dp_last_error_detail(void) { return g_detail; }
+
+dp_status dp_set_device(int32_t ordinal) {
+  cudaError_t e = cudaSetDevice(ordinal);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  return DP_OK;
+}
+
+dp_status dp_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t word = 0;
+  e = cudaMemcpyFromSymbol(&word, dp_status_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (word) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(dp_status_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+    return fail(DP_ERR_TIMEOUT, "device wait gave up (status word 0x%x)", word);
+  }
+  return DP_OK;
+}
+
+dp_status dp_blocks_from_table(dp_blocks* out, const float* table, int32_t table_rows, int32_t hidden,
+                               const int32_t* timesteps, const int32_t* block_rows, int32_t n_blocks) {
+  if (!out || !table || !timesteps || !block_rows) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  if (n_blocks < 1 || n_blocks > DP_MAX_BLOCKS) return fail(DP_ERR_INVALID_ARG, "n_blocks %d", n_blocks);
+  if (hidden <= 0 || hidden % 4) return fail(DP_ERR_INVALID_ARG, "hidden %d", hidden);
+  if (!aligned16(table)) return fail(DP_ERR_INVALID_ARG, "table misaligned");
+  dp_blocks b;
+  memset(&b, 0, sizeof(b));
+  b.n_blocks = n_blocks;
+  b.hidden = hidden;
+  int64_t off = 0;
+  for (int i = 0; i < n_blocks; ++i) {
+    if (timesteps[i] < 0 || timesteps[i] >= table_rows)
+      return fail(DP_ERR_INVALID_ARG, "timestep %d outside [0, %d)", timesteps[i], table_rows);
+    if (block_rows[i] < 0) return fail(DP_ERR_INVALID_ARG, "block_rows[%d] negative", i);
+    b.row_offset[i] = static_cast<int32_t>(off);
+    off += block_rows[i];
+    if (off > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "window rows overflow");
+    b.mod[i] = table + static_cast<int64_t>(timesteps[i]) * 3 * hidden;
+  }
+  b.row_offset[n_blocks] = static_cast<int32_t>(off);
+  *out = b;
+  return DP_OK;
+}
+
+dp_status dp_queue_blocks(const dp_queue* q, const float* table, int32_t table_rows, const int32_t* tau, int32_t n_tau,
+                          dp_blocks* out, const void** window, int64_t* n_win) {
+  if (!q || !table || !tau || !out || !window || !n_win) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  dp_status st = check_queue(q, q->hidden, q->dtype);
+  if (st != DP_OK) return st;
+  if (q->count == 0) return fail(DP_ERR_EMPTY, "queue is empty");
+  int32_t ts[DP_MAX_SLOTS];
+  for (int i = 0; i < q->count; ++i) {
+    if (q->evals[i] < 0 || q->evals[i] >= n_tau)
+      return fail(DP_ERR_INVALID_ARG, "block %d has had %d evaluations of %d", i, q->evals[i], n_tau);
+    ts[i] = tau[q->evals[i]];
+  }
+  st = dp_blocks_from_table(out, table, table_rows, q->hidden, ts, q->rows, q->count);
+  if (st != DP_OK) return st;
+  *window = queue_slot(q, q->head);
+  *n_win = out->row_offset[q->count];
+  return DP_OK;
+}
+
+dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blocks* blk, dp_dtype dt, void* stream) {
+  if (!dtype_ok(dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return fail(DP_ERR_INVALID_ARG, "x/y NULL or misaligned");
+  if (n_rows <= 0) return fail(DP_ERR_INVALID_ARG, "n_rows %lld", static_cast<long long>(n_rows));
+  if (!blk) return fail(DP_ERR_INVALID_ARG, "block table is NULL");
+  if (!hidden_ok(blk->hidden, dt)) return fail(DP_ERR_INVALID_ARG, "hidden %d not a whole number of 16-byte vectors", blk->hidden);
+  dp_status st = check_blocks(blk, n_rows, blk->hidden);
+  if (st != DP_OK) return st;
+  const dp::BlockTable t = to_table(blk);
+  const void* src[1] = {x};
+  void* dst[1] = {y};
+  cudaError_t e = dp::launch_modulate(src, dst, 1, n_rows, blk->hidden, t, dt, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
+  return DP_OK;
+}
+
+namespace {
+
+dp_status check_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* ck, const void* cv,
+                          int64_t cache_len, const void* residual, void* out, int32_t n_heads, int32_t head_dim,
+                          const dp_blocks* blk, dp_dtype dt) {
+  if (!dtype_ok(dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+  if (!q || !k || !v || !out) return fail(DP_ERR_INVALID_ARG, "q/k/v/out NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (residual && !aligned16(residual)))
+    return fail(DP_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+  if (n_win <= 0 || n_win > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_win %lld", static_cast<long long>(n_win));
+  if (cache_len < 0 || cache_len > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "cache_len %lld", static_cast<long long>(cache_len));
+  if (cache_len > 0 && (!ck || !cv || !aligned16(ck) || !aligned16(cv)))
+    return fail(DP_ERR_INVALID_ARG, "cache k/v NULL or misaligned");
+  if (n_heads <= 0 || head_dim <= 0) return fail(DP_ERR_INVALID_ARG, "n_heads/head_dim");
+  const int64_t hidden = static_cast<int64_t>(n_heads) * head_dim;
+  if (hidden > INT32_MAX || !hidden_ok(static_cast<int32_t>(hidden), dt)) return fail(DP_ERR_INVALID_ARG, "hidden");
+  if (dt == DP_BF16 && head_dim != 64 && head_dim != 128)
+    return fail(DP_ERR_UNSUPPORTED, "bf16 head_dim %d (64 or 128 supported)", head_dim);
+  if (dt == DP_F32 && head_dim != 4 && head_dim != 8 && head_dim != 16 && head_dim != 32 && head_dim != 64 &&
+      head_dim != 128)
+    return fail(DP_ERR_UNSUPPORTED, "f32 head_dim %d (4, 8, 16, 32, 64 or 128 supported)", head_dim);
+  if (out == q || out == k || out == v || (residual && out == residual) || (cache_len > 0 && (out == ck || out == cv)))
+    return fail(DP_ERR_INVALID_ARG, "out aliases an input");
+  return check_blocks(blk, n_win, static_cast<int32_t>(hidden));
+}
+
+dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* ck, const void* cv,
+                        int64_t cache_len, const void* residual, void* out, int32_t n_heads, int32_t head_dim,
+                        float softmax_scale, const dp_blocks* blk, uint32_t flags, dp_dtype dt, cudaStream_t s) {
+  dp::AttnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cache_k = ck;
+  a.cache_v = cv;
+  a.residual = residual;
+  a.out = out;
+  a.n_win = n_win;
+  a.cache_len = cache_len;
+  a.n_heads = n_heads;
+  a.head_dim = head_dim;
+  a.hidden = n_heads * head_dim;
+  a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(head_dim));
+  a.flags = flags;
+  a.bt = to_table(blk);
+  dp_status st = status_ptr(&a.status);
+  if (st != DP_OK) return st;
+  cudaError_t e = dt == DP_BF16 ? dp::launch_attention_bf16(a, s) : dp::launch_attention_f32(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return DP_OK;
+}
+
+}  // namespace
+
+dp_status dp_window_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* cache_k,
+                              const void* cache_v, int64_t cache_len, const void* residual, void* out,
+                              int32_t n_heads, int32_t head_dim, float softmax_scale, const dp_blocks* blk,
+                              uint32_t flags, dp_dtype dt, void* stream) {
+  dp_status st = check_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, blk, dt);
+  if (st != DP_OK) return st;
+  return run_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, softmax_scale,
+                       blk, flags, dt, static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_kvcache_advance(dp_kvcache* c, const void* k_exit, const void* v_exit, int64_t n_exit, void* stream) {
+  if (!c) return fail(DP_ERR_INVALID_ARG, "cache is NULL");
+  dp_status st = check_cache(c, c->hidden, c->dtype);
+  if (st != DP_OK) return st;
+  if (!hidden_ok(c->hidden, c->dtype)) return fail(DP_ERR_INVALID_ARG, "hidden");
+  if (n_exit < 0) return fail(DP_ERR_INVALID_ARG, "n_exit negative");
+  if (n_exit > c->capacity)
+    return fail(DP_ERR_CAPACITY, "exiting block of %lld rows > cache capacity %lld", static_cast<long long>(n_exit),
+                static_cast<long long>(c->capacity));
+  if (n_exit > 0 && (!k_exit || !v_exit || !aligned16(k_exit) || !aligned16(v_exit)))
+    return fail(DP_ERR_INVALID_ARG, "k_exit/v_exit NULL or misaligned");
+  const int64_t row_bytes = static_cast<int64_t>(c->hidden) * elem_bytes(c->dtype);
+  const int64_t slot = c->n_advances % c->n_slots;
+  dp::CopySeg segs[2] = {
+      {k_exit, static_cast<char*>(c->k) + slot * c->capacity * row_bytes, n_exit * row_bytes},
+      {v_exit, static_cast<char*>(c->v) + slot * c->capacity * row_bytes, n_exit * row_bytes}};
+  cudaError_t e = dp::launch_copy(segs, 2, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "advance copy");
+  c->len[slot] = n_exit;
+  c->n_advances += 1;
+  return DP_OK;
+}
+
+dp_status dp_queue_push(dp_queue* q, const void* noise, int64_t rows, void* stream) {
+  if (!q) return fail(DP_ERR_INVALID_ARG, "queue is NULL");
+  dp_status st = check_queue(q, q->hidden, q->dtype);
+  if (st != DP_OK) return st;
+  st = check_push(q, q->count, noise, rows);
+  if (st != DP_OK) return st;
+  const int64_t bytes = rows * q->hidden * elem_bytes(q->dtype);
+  const int32_t p = (q->head + q->count) % q->n_slots;
+  dp::CopySeg segs[2] = {{noise, queue_slot(q, p), bytes}, {noise, queue_slot(q, p + q->n_slots), bytes}};
+  cudaError_t e = dp::launch_copy(segs, 2, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "push copy");
+  apply_push(q, rows);
+  return DP_OK;
+}
+
+dp_status dp_queue_pop(dp_queue* q) {
+  if (!q) return fail(DP_ERR_INVALID_ARG, "queue is NULL");
+  dp_status st = check_queue(q, q->hidden, q->dtype);
+  if (st != DP_OK) return st;
+  if (q->count == 0) return fail(DP_ERR_EMPTY, "queue is empty");
+  apply_pop(q);
+  return DP_OK;
+}
+
+dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_win, const dp_blocks* blk,
+                         dp_kvcache* cache, void* kv_work, const void* residual, void* out, int32_t n_heads,
+                         int32_t head_dim, uint32_t flags, dp_queue* queue, const void* push_noise, int64_t push_rows,
+                         dp_dtype dt, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!cache) return fail(DP_ERR_INVALID_ARG, "cache is NULL");
+  const int64_t hidden64 = static_cast<int64_t>(n_heads) * head_dim;
+  if (n_heads <= 0 || head_dim <= 0 || hidden64 > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_heads/head_dim");
+  const int32_t hidden = static_cast<int32_t>(hidden64);
+  dp_status st = check_cache(cache, hidden, dt);
+  if (st != DP_OK) return st;
+  if (!kv_work || !aligned16(kv_work)) return fail(DP_ERR_INVALID_ARG, "kv_work NULL or misaligned");
+  const int64_t rslot = cache_read_slot(cache);
+  const int64_t row_bytes = hidden64 * elem_bytes(dt);
+  const char* ck = static_cast<const char*>(cache->k) + rslot * cache->capacity * row_bytes;
+  const char* cv = static_cast<const char*>(cache->v) + rslot * cache->capacity * row_bytes;
+  const int64_t cache_len = cache->len[rslot];
+  char* kp = static_cast<char*>(kv_work);
+  char* vp = kp + n_win * row_bytes;
+  st = check_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, blk, dt);
+  if (st != DP_OK) return st;
+  if (out == kv_work) return fail(DP_ERR_INVALID_ARG, "out aliases kv_work");
+  const bool pop = (flags & DP_STEP_POP) != 0;
+  const int64_t n_exit = blk->row_offset[1];
+  if (pop && n_exit > cache->capacity)
+    return fail(DP_ERR_CAPACITY, "head block of %lld rows > cache capacity", static_cast<long long>(n_exit));
+  if (queue) {
+    st = check_queue(queue, hidden, dt);
+    if (st != DP_OK) return st;
+    if (pop && queue->count == 0) return fail(DP_ERR_EMPTY, "pop from an empty queue");
+  }
+  if (push_noise) {
+    if (!queue) return fail(DP_ERR_INVALID_ARG, "push needs a queue");
+    st = check_push(queue, queue->count - (pop ? 1 : 0), push_noise, push_rows);
+    if (st != DP_OK) return st;
+  }
+
+  // A1: k' and v' of the window (one launch, two segments)
+  const dp::BlockTable t = to_table(blk);
+  const void* src[2] = {k, v};
+  void* dst[2] = {kp, vp};
+  cudaError_t e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, s);
+  if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
+  // A2: attention with the Q prologue and gate epilogue
+  st = run_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, 0.0f, blk,
+                     DP_MOD_Q | DP_GATE_OUT, dt, s);
+  if (st != DP_OK) return st;
+  // A3: pop (head block's k'/v' -> cache ring) and push (noise -> latent ring), one launch.
+  // Descriptors change only after the launch has been accepted.
+  dp::CopySeg segs[dp::kMaxCopySegs];
+  int nseg = 0;
+  const int64_t wslot = cache->n_advances % cache->n_slots;
+  if (pop) {
+    segs[nseg++] = {kp, static_cast<char*>(cache->k) + wslot * cache->capacity * row_bytes, n_exit * row_bytes};
+    segs[nseg++] = {vp, static_cast<char*>(cache->v) + wslot * cache->capacity * row_bytes, n_exit * row_bytes};
+  }
+  if (push_noise) {
+    const int32_t head_after = (queue->head + ((pop && queue) ? 1 : 0)) % queue->n_slots;
+    const int32_t count_after = queue->count - (pop ? 1 : 0);
+    const int32_t p = (head_after + count_after) % queue->n_slots;
+    const int64_t bytes = push_rows * row_bytes;
+    segs[nseg++] = {push_noise, queue_slot(queue, p), bytes};
+    segs[nseg++] = {push_noise, queue_slot(queue, p + queue->n_slots), bytes};
+  }
+  if (nseg) {
+    e = dp::launch_copy(segs, nseg, s);
+    if (e != cudaSuccess) return cuda_fail(e, "advance copy");
+  }
+  if (queue)
+    for (int i = 0; i < queue->count; ++i) queue->evals[i] += 1;
+  if (pop) {
+    cache->len[wslot] = n_exit;
+    cache->n_advances += 1;
+    if (queue) apply_pop(queue);
+  }
+  if (push_noise) apply_push(queue, push_rows);
+  return DP_OK;
+}
+
+}  // extern "C"

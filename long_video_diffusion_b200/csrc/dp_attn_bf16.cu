@@ -1,0 +1,523 @@
+// Window attention over [cached K/V ; window K/V] on the sm_100a tensor cores.
+//
+// Operation ("Minute-Long Videos with Dual Parallelisms", abstract: the feature cache of
+// the prior block is reused as context; pith.science review, Section 3.2: self-attention
+// over the cached K/V of the neighbouring block plus the block's own K/V):
+//   q'_i = q_i * (1 + scale_b) + shift_b            (prologue, b = block of row i)
+//   o_i  = softmax_j(q'_i . K_j * scale) V_j         (j: cache rows, then window rows)
+//   out_i = gate_b * o_i (+ residual_i)              (epilogue)
+//
+// Design (one CTA = two 128-row query tiles of one head; keys in 128-row tiles):
+//   warps 0-3  softmax warpgroup for query tile 0 (one thread per query row)
+//   warps 4-7  softmax warpgroup for query tile 1
+//   warp 8     TMA producer: K and V tiles into a ring of shared-memory stages
+//   warp 9     TMEM owner and MMA issuer (one thread issues tcgen05.mma)
+//   warps 10-11 idle (they complete the third warpgroup, which setmaxnreg needs)
+// Registers: launched at kLaunchRegs per thread; the producer warpgroup gives registers
+// back (kLowRegs) and the two softmax warpgroups take them (kHighRegs), so a softmax
+// thread can hold its 128 scores without spilling.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+HD), O1 after it.
+// P (bf16) is written over the first 64 columns of its S tile and consumed from TMEM as
+// the A operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both
+// K-major with the 128-byte swizzle; V is the MN-major B operand of the PV product.
+// Softmax is fp32 with exp2 on the MUFU unit; the running max is only moved (and O
+// rescaled) when it grows by more than 2^8, which keeps the result exact because the
+// final 1/l uses the same reference max as the numerator.
+// Every wait is bounded (see dp_device.cuh): on giving up the kernel records a timeout in
+// the device status word, stops issuing work, drains its own copies and MMAs, frees TMEM
+// and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+
+#include "dp_device.cuh"
+#include "dp_internal.h"
+
+namespace dp {
+
+namespace {
+
+constexpr int BM = 128;       // query rows per tile
+constexpr int BN = 128;       // keys per tile
+constexpr int NQ = 2;         // query tiles per CTA
+constexpr int kThreads = 384; // 12 warps
+constexpr int kLaunchRegs = 168;  // 65536 / 384 rounded down to the allocation granule
+constexpr int kLowRegs = 72;
+constexpr int kHighRegs = 216;
+static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
+constexpr int kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
+
+template <int HD>
+struct Layout {
+  static constexpr int KCH = HD / 64;                    // 128-byte column chunks
+  static constexpr int STAGES = (HD == 64) ? 4 : 2;
+  static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 B
+  static constexpr int Q_BYTES = BM * HD * 2;
+  static constexpr int KV_BYTES = BN * HD * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  // k_full[S], v_full[S], kv_empty[S], q_full[2], s_full[2], p_full[2], o_done[2], fin
+  static constexpr int N_BAR = 3 * STAGES + 4 * NQ + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;             // room to align the base to 1 KB
+  static_assert(ALLOC <= 227 * 1024, "shared memory budget");
+  static_assert(256 + NQ * HD <= kTmemCols, "tensor memory budget");
+};
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* out;
+  int64_t n_win;
+  int64_t cache_len;
+  int32_t hidden;
+  int32_t n_qpairs;
+  int32_t n_ct;  // cache key tiles
+  int32_t n_wt;  // window key tiles
+  float scale_log2;
+  uint32_t flags;
+  uint32_t* status;
+  BlockTable bt;
+};
+
+// Bounded wait that ignores the abort flag: used to drain work this CTA already issued.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(status, DEV_ERR_TIMEOUT_DRAIN);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+                     const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
+                     const Params p) {
+  using L = Layout<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qpair = blockIdx.x % p.n_qpairs;   // consecutive CTAs share a head (K/V reuse in L2)
+  const int head = blockIdx.x / p.n_qpairs;
+  const int n_tiles = p.n_ct + p.n_wt;
+
+  const uint32_t bar0 = sb + L::OFF_BAR;
+  auto k_full = [&](int s) { return bar0 + 8u * s; };
+  auto v_full = [&](int s) { return bar0 + 8u * (L::STAGES + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 * L::STAGES + s); };
+  auto q_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + g); };
+  auto s_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + NQ + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 2 * NQ + g); };
+  auto o_done = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 3 * NQ + g); };
+  const uint32_t fin = bar0 + 8u * (3 * L::STAGES + 4 * NQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int g = 0; g < NQ; ++g) {
+      mbar_init(q_full(g), 128);
+      mbar_init(s_full(g), 1);
+      mbar_init(p_full(g), 128);
+      mbar_init(o_done(g), 1);
+    }
+    mbar_init(fin, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_kc);
+    tma_prefetch_desc(&tm_vc);
+    tma_prefetch_desc(&tm_kw);
+    tma_prefetch_desc(&tm_vw);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % L::STAGES;
+        const int use = j / L::STAGES;
+        if (use > 0 && !mbar_wait(kv_empty(st), (use - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_EMPTY)) break;
+        const bool cache = j < p.n_ct;
+        const CUtensorMap* mk = cache ? &tm_kc : &tm_kw;
+        const CUtensorMap* mv = cache ? &tm_vc : &tm_vw;
+        const int row = (cache ? j : j - p.n_ct) * BN;
+        mbar_arrive_expect_tx(k_full(st), L::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_2d(sb + L::OFF_K + st * L::KV_BYTES + c * L::CHUNK_BYTES, mk, head * HD + c * 64, row, k_full(st));
+        mbar_arrive_expect_tx(v_full(st), L::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < L::KCH; ++c)
+          tma_load_2d(sb + L::OFF_V + st * L::KV_BYTES + c * L::CHUNK_BYTES, mv, head * HD + c * 64, row, v_full(st));
+        issued = j + 1;
+      }
+      // every copy this CTA issued must land before its shared memory is released
+      const int first = issued > L::STAGES ? issued - L::STAGES : 0;
+      for (int j = first; j < issued; ++j) {
+        drain_wait(k_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
+        drain_wait(v_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, true);
+      auto issue_s = [&](int g, int st) {
+        const uint32_t qa = sb + L::OFF_Q + g * L::Q_BYTES;
+        const uint32_t ka = sb + L::OFF_K + st * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + g * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int g, int st, bool acc) {
+        const uint32_t va = sb + L::OFF_V + st * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          mma_ts(tmem + 256 + g * HD, tmem + g * 128 + kk * 8, sdesc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), idPV,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full(0), 0, abort, p.status, DEV_ERR_TIMEOUT_Q) &&
+                mbar_wait(q_full(1), 0, abort, p.status, DEV_ERR_TIMEOUT_Q) &&
+                mbar_wait(k_full(0), 0, abort, p.status, DEV_ERR_TIMEOUT_KV);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(s_full(0));
+        issue_s(1, 0);
+        mma_commit(s_full(1));
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % L::STAGES;
+        if (!mbar_wait(v_full(st), (j / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV)) break;
+        for (int g = 0; g < NQ && ok; ++g) {
+          if (!mbar_wait(p_full(g), j & 1, abort, p.status, DEV_ERR_TIMEOUT_P)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(g, st, j > 0);
+          mma_commit(o_done(g));
+          if (g == NQ - 1) mma_commit(kv_empty(st));
+          if (j + 1 < n_tiles) {
+            const int st1 = (j + 1) % L::STAGES;
+            if (g == 0) {
+              if (!mbar_wait(k_full(st1), ((j + 1) / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            // S(g) of the next tile overwrites P(g) of this tile: the MMAs issued by this
+            // thread execute in issue order, so the PV product above has read P first.
+            issue_s(g, st1);
+            mma_commit(s_full(g));
+          }
+        }
+      }
+      mma_commit(fin);
+      drain_wait(fin, 0, p.status);
+    }
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    // ------------------------------------------------------------ softmax warpgroups
+    const int g = warp >> 2;                       // query tile of this warpgroup
+    const int t = threadIdx.x & 127;               // row within the tile
+    const int64_t qrow = static_cast<int64_t>(qpair) * (NQ * BM) + g * BM + t;
+    const bool row_ok = qrow < p.n_win;
+    const int blk = row_ok ? block_of_row(p.bt, qrow) : 0;
+    const float* modb = block_mod(p.bt, blk);
+
+    // prologue: modulated query row -> swizzled K-major shared-memory tile
+    {
+      uint8_t* sq = smem + L::OFF_Q + g * L::Q_BYTES;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + qrow * p.hidden + head * HD);
+      const float* shift = modb + head * HD;
+      const float* scale = modb + p.hidden + head * HD;
+#pragma unroll 4
+      for (int c = 0; c < HD / 8; ++c) {
+        uint4 outv = make_uint4(0, 0, 0, 0);
+        if (row_ok) {
+          uint4 raw = src[c];
+          if (p.flags & DP_MOD_Q) {
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            const float4 sh0 = ld_f4(shift + c * 8), sh1 = ld_f4(shift + c * 8 + 4);
+            const float4 sc0 = ld_f4(scale + c * 8), sc1 = ld_f4(scale + c * 8 + 4);
+            const float sh[8] = {sh0.x, sh0.y, sh0.z, sh0.w, sh1.x, sh1.y, sh1.z, sh1.w};
+            const float sc[8] = {sc0.x, sc0.y, sc0.z, sc0.w, sc1.x, sc1.y, sc1.z, sc1.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = __bfloat1622float2(x2[e]);
+              o[e] = pack_bf16x2(fmaf(xf.x, 1.0f + sc[2 * e], sh[2 * e]), fmaf(xf.y, 1.0f + sc[2 * e + 1], sh[2 * e + 1]));
+            }
+            outv = make_uint4(o[0], o[1], o[2], o[3]);
+          } else {
+            outv = raw;
+          }
+        }
+        const int chunk = c >> 3, w = c & 7;
+        *reinterpret_cast<uint4*>(sq + chunk * L::CHUNK_BYTES + t * 128 + ((w ^ (t & 7)) << 4)) = outv;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_full(g));
+    }
+
+    const uint32_t trow = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
+    const uint32_t s_col = g * 128;
+    const uint32_t o_col = 256 + g * HD;
+    float m_ref = -INFINITY;
+    float l_sum = 0.0f;
+    bool ok = true;
+
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = mbar_wait(s_full(g), j & 1, abort, p.status, DEV_ERR_TIMEOUT_S);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(trow + s_col + i * 32, sr[i]);
+      tmem_wait_ld();
+      const int64_t key0 = (j < p.n_ct) ? static_cast<int64_t>(j) * BN : static_cast<int64_t>(j - p.n_ct) * BN;
+      const int64_t seg_len = (j < p.n_ct) ? p.cache_len : p.n_win;
+      const int64_t rem = seg_len - key0;
+      const int valid = rem < BN ? static_cast<int>(rem) : BN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (i * 32 + c >= valid) sr[i][c] = 0xff800000u;  // -inf: key beyond the segment
+          mx = fmaxf(mx, __uint_as_float(sr[i][c]));
+        }
+      }
+      const float m_new = fmaxf(m_ref, mx * p.scale_log2);
+      if (j == 0) {
+        m_ref = m_new;
+      } else {
+        const bool need = m_new > m_ref + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          // the previous PV product must be complete before O is read and rescaled
+          ok = mbar_wait(o_done(g), (j - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
+#pragma unroll
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t orr[32];
+            tmem_ld32(trow + o_col + c0, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * f);
+            tmem_st32(trow + o_col + c0, orr);
+          }
+          tmem_wait_st();
+          if (need) {
+            l_sum *= f;
+            m_ref = m_new;
+          }
+        }
+      }
+      const float nm = -m_ref;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float a = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c]), p.scale_log2, nm));
+          const float b = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c + 1]), p.scale_log2, nm));
+          l_sum += a + b;
+          pk[c] = pack_bf16x2(a, b);
+        }
+        tmem_st16(trow + s_col + i * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(g));
+    }
+
+    // epilogue: O / l, gate, residual, bf16 store
+    if (ok && n_tiles > 0) {
+      ok = mbar_wait(o_done(g), (n_tiles - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_sum;
+      const float* gate = modb + 2 * p.hidden + head * HD;
+      const bool do_gate = (p.flags & DP_GATE_OUT) != 0;
+#pragma unroll
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t orr[32];
+        tmem_ld32(trow + o_col + c0, orr);
+        tmem_wait_ld();
+        if (row_ok) {
+          float vals[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) vals[c] = __uint_as_float(orr[c]) * inv_l;
+          if (do_gate) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              const float4 gv = ld_f4(gate + c0 + c);
+              vals[c] *= gv.x;
+              vals[c + 1] *= gv.y;
+              vals[c + 2] *= gv.z;
+              vals[c + 3] *= gv.w;
+            }
+          }
+          if (p.residual) {
+            const uint4* rs = reinterpret_cast<const uint4*>(p.residual + qrow * p.hidden + head * HD + c0);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint4 r = rs[c];
+              const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 rf = __bfloat1622float2(r2[e]);
+                vals[c * 8 + 2 * e] += rf.x;
+                vals[c * 8 + 2 * e + 1] += rf.y;
+              }
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.out + qrow * p.hidden + head * HD + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            dst[c] = make_uint4(pack_bf16x2(vals[c * 8 + 0], vals[c * 8 + 1]), pack_bf16x2(vals[c * 8 + 2], vals[c * 8 + 3]),
+                                pack_bf16x2(vals[c * 8 + 4], vals[c * 8 + 5]), pack_bf16x2(vals[c * 8 + 6], vals[c * 8 + 7]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+template <int HD>
+cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
+  using L = Layout<HD>;
+  CUtensorMap tkc, tvc, tkw, tvw;
+  if (!encode_tmap_bf16(&tkw, a.k, a.n_win, a.hidden) || !encode_tmap_bf16(&tvw, a.v, a.n_win, a.hidden))
+    return cudaErrorInvalidValue;
+  if (a.cache_len > 0) {
+    if (!encode_tmap_bf16(&tkc, a.cache_k, a.cache_len, a.hidden) ||
+        !encode_tmap_bf16(&tvc, a.cache_v, a.cache_len, a.hidden))
+      return cudaErrorInvalidValue;
+  } else {
+    tkc = tkw;
+    tvc = tvw;
+  }
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.residual = static_cast<const __nv_bfloat16*>(a.residual);
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.n_win = a.n_win;
+  p.cache_len = a.cache_len;
+  p.hidden = a.hidden;
+  p.n_qpairs = static_cast<int32_t>((a.n_win + NQ * BM - 1) / (NQ * BM));
+  p.n_ct = static_cast<int32_t>((a.cache_len + BN - 1) / BN);
+  p.n_wt = static_cast<int32_t>((a.n_win + BN - 1) / BN);
+  p.scale_log2 = a.softmax_scale * 1.4426950408889634f;
+  p.flags = a.flags;
+  p.status = a.status;
+  p.bt = a.bt;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(attn_bf16_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    // setmaxnreg.inc waits for registers the launch did not provide: refuse to launch if
+    // the compiled register count is below the split's assumption.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_bf16_kernel<HD>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+    attr_set[dev] = true;
+  }
+  const int64_t grid = static_cast<int64_t>(p.n_qpairs) * a.n_heads;
+  attn_bf16_kernel<HD><<<static_cast<unsigned>(grid), kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool encode_tmap_bf16(void* tmap, const void* base, int64_t rows, int hidden) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(hidden) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(static_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
+  if (a.head_dim == 64) return launch_hd<64>(a, s);
+  if (a.head_dim == 128) return launch_hd<128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dp

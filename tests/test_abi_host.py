@@ -1,0 +1,200 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls): the library loads and
+exports every entry point include/dp.h declares, the ctypes mirrors match the C struct
+layouts, and argument errors are reported synchronously before anything is enqueued."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dp.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:dp_status|const char\*|int32_t)\s+(dp_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def m():
+    import long_video_diffusion_b200 as mod
+    return mod
+
+
+def test_library_exports_every_declared_function(m):
+    declared = _declared_functions()
+    assert len(declared) >= 13
+    out = subprocess.run(["nm", "-D", "--defined-only", m.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dp_\w+)$", out, flags=re.M))
+    missing = [f for f in declared if f not in exported]
+    assert not missing, missing
+    assert sorted(m.EXPORTS) == declared
+    for f in declared:
+        assert hasattr(m._lib, f)
+    assert m.version() == 100
+
+
+def test_status_strings(m):
+    for code, name in [(0, "DP_OK"), (-1, "DP_ERR_INVALID_ARG"), (-5, "DP_ERR_TIMEOUT"), (-6, "DP_ERR_EMPTY")]:
+        assert m._lib.dp_status_string(code).decode() == name
+
+
+def test_ctypes_layouts_match_c(tmp_path, m):
+    src = tmp_path / "layout.c"
+    src.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "dp.h"
+int main(void) {
+  printf("%zu %zu %zu\\n", sizeof(dp_blocks), offsetof(dp_blocks, row_offset), offsetof(dp_blocks, mod));
+  printf("%zu %zu %zu %zu\\n", sizeof(dp_kvcache), offsetof(dp_kvcache, len), offsetof(dp_kvcache, n_advances),
+         offsetof(dp_kvcache, dtype));
+  printf("%zu %zu %zu %zu\\n", sizeof(dp_queue), offsetof(dp_queue, rows), offsetof(dp_queue, n_pushed),
+         offsetof(dp_queue, dtype));
+  return 0;
+}
+""")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    lines = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    b = [int(x) for x in lines[0].split()]
+    c = [int(x) for x in lines[1].split()]
+    q = [int(x) for x in lines[2].split()]
+    assert b == [ctypes.sizeof(m.DpBlocks), m.DpBlocks.row_offset.offset, m.DpBlocks.mod.offset]
+    assert c == [ctypes.sizeof(m.DpKvcache), m.DpKvcache.len.offset, m.DpKvcache.n_advances.offset,
+                 m.DpKvcache.dtype.offset]
+    assert q == [ctypes.sizeof(m.DpQueue), m.DpQueue.rows.offset, m.DpQueue.n_pushed.offset,
+                 m.DpQueue.dtype.offset]
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned, never dereferenced: every call below fails its checks first
+
+
+def _blocks(m, rows, hidden):
+    b = m.DpBlocks()
+    b.n_blocks = len(rows)
+    b.hidden = hidden
+    off = 0
+    for i, r in enumerate(rows):
+        b.row_offset[i] = off
+        b.mod[i] = FAKE + 4096 * i
+        off += r
+    b.row_offset[len(rows)] = off
+    return b
+
+
+def test_blocks_from_table_checks(m):
+    out = m.DpBlocks()
+    ts = (ctypes.c_int32 * 2)(0, 1000)
+    rows = (ctypes.c_int32 * 2)(4, 4)
+    assert m._lib.dp_blocks_from_table(ctypes.byref(out), ctypes.c_void_p(FAKE), 1000, 64, ts, rows, 2) == m.ERR_INVALID_ARG
+    ts = (ctypes.c_int32 * 2)(0, 999)
+    assert m._lib.dp_blocks_from_table(ctypes.byref(out), ctypes.c_void_p(FAKE), 1000, 64, ts, rows, 2) == m.OK
+    assert out.offsets == [0, 4, 8]
+    assert out.mod[1] == FAKE + 999 * 3 * 64 * 4
+    assert m._lib.dp_blocks_from_table(ctypes.byref(out), ctypes.c_void_p(FAKE), 1000, 64, ts, rows, 17) == m.ERR_INVALID_ARG
+
+
+def _attn(m, q=FAKE, k=FAKE + 1024, v=FAKE + 2048, n=256, ck=FAKE + 4096, cv=FAKE + 8192, lc=128,
+          out=FAKE + 16384, H=2, hd=64, blk=None, dt=1):
+    blk = blk if blk is not None else _blocks(m, [128, 128], H * hd)
+    return m._lib.dp_window_attention(ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v), n,
+                                      ctypes.c_void_p(ck), ctypes.c_void_p(cv), lc, None, ctypes.c_void_p(out),
+                                      H, hd, 0.0, ctypes.byref(blk), 3, dt, None)
+
+
+def test_attention_argument_errors(m):
+    assert _attn(m, q=0) == m.ERR_INVALID_ARG                       # NULL
+    assert _attn(m, q=FAKE + 8) == m.ERR_INVALID_ARG                # misaligned
+    assert _attn(m, n=0, blk=_blocks(m, [0], 128)) == m.ERR_INVALID_ARG
+    assert _attn(m, H=1, hd=96, blk=_blocks(m, [128, 128], 96)) == m.ERR_UNSUPPORTED
+    assert _attn(m, H=1, hd=96, dt=0, blk=_blocks(m, [128, 128], 96)) == m.ERR_UNSUPPORTED
+    assert _attn(m, blk=_blocks(m, [128, 127], 128)) == m.ERR_INVALID_ARG   # offsets != n_win
+    assert _attn(m, out=FAKE) == m.ERR_INVALID_ARG                  # out aliases q
+    assert _attn(m, lc=-1) == m.ERR_INVALID_ARG
+    assert _attn(m, ck=0, lc=5) == m.ERR_INVALID_ARG
+    bad = _blocks(m, [128, 128], 128)
+    bad.mod[1] = 0
+    assert _attn(m, blk=bad) == m.ERR_INVALID_ARG
+    assert b"mod[1]" in m._lib.dp_last_error_detail()
+    assert _attn(m, dt=7) == m.ERR_INVALID_ARG
+
+
+def _cache(m, capacity=128, hidden=128, n_slots=1, length=0, dt=1):
+    c = m.DpKvcache()
+    c.k, c.v = FAKE + (1 << 20), FAKE + (2 << 20)
+    c.capacity, c.hidden, c.n_slots, c.dtype = capacity, hidden, n_slots, dt
+    c.len[0] = length
+    return c
+
+
+def test_advance_capacity_errors(m):
+    c = _cache(m)
+    assert m._lib.dp_kvcache_advance(ctypes.byref(c), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), 129, None) == m.ERR_CAPACITY
+    assert c.n_advances == 0
+    c.len[0] = 200
+    assert m._lib.dp_kvcache_advance(ctypes.byref(c), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), 1, None) == m.ERR_CAPACITY
+
+
+def _queue(m, n_slots=2, slot_rows=64, hidden=128, count=0, rows=(), dt=1):
+    q = m.DpQueue()
+    q.latent = FAKE + (8 << 20)
+    q.slot_rows, q.hidden, q.n_slots, q.count, q.dtype = slot_rows, hidden, n_slots, count, dt
+    for i, r in enumerate(rows):
+        q.rows[i] = r
+    return q
+
+
+def test_queue_host_logic(m):
+    q = _queue(m)
+    assert m._lib.dp_queue_pop(ctypes.byref(q)) == m.ERR_EMPTY
+    full = _queue(m, count=2, rows=(64, 64))
+    assert m._lib.dp_queue_push(ctypes.byref(full), ctypes.c_void_p(FAKE), 64, None) == m.ERR_CAPACITY
+    short = _queue(m, n_slots=3, count=1, rows=(32,))
+    assert m._lib.dp_queue_push(ctypes.byref(short), ctypes.c_void_p(FAKE), 64, None) == m.ERR_INVALID_ARG
+    big = _queue(m, n_slots=3)
+    assert m._lib.dp_queue_push(ctypes.byref(big), ctypes.c_void_p(FAKE), 65, None) == m.ERR_CAPACITY
+    # pop is metadata only: head rotates, rows/evals shift toward the head
+    q = _queue(m, n_slots=3, count=3, rows=(64, 64, 40))
+    q.head = 2
+    q.evals[0], q.evals[1], q.evals[2] = 9, 5, 1
+    assert m._lib.dp_queue_pop(ctypes.byref(q)) == m.OK
+    assert (q.head, q.count, q.n_popped) == (0, 2, 1)
+    assert [q.rows[i] for i in range(2)] == [64, 40] and [q.evals[i] for i in range(2)] == [5, 1]
+
+
+def test_queue_blocks_host_lookup(m):
+    q = _queue(m, n_slots=4, slot_rows=64, count=3, rows=(64, 64, 16))
+    q.head = 3
+    q.evals[0], q.evals[1], q.evals[2] = 4, 2, 0
+    tau = (ctypes.c_int32 * 5)(999, 750, 500, 250, 0)
+    out = m.DpBlocks()
+    win = ctypes.c_void_p()
+    n = ctypes.c_int64()
+    assert m._lib.dp_queue_blocks(ctypes.byref(q), ctypes.c_void_p(FAKE), 1000, tau, 5, ctypes.byref(out),
+                                  ctypes.byref(win), ctypes.byref(n)) == m.OK
+    assert n.value == 144 and out.offsets == [0, 64, 128, 144]
+    assert win.value == FAKE + (8 << 20) + 3 * 64 * 128 * 2          # head slot of the mirrored ring
+    assert [out.mod[i] for i in range(3)] == [FAKE + t * 3 * 128 * 4 for t in (0, 500, 999)]
+    q.evals[0] = 5
+    assert m._lib.dp_queue_blocks(ctypes.byref(q), ctypes.c_void_p(FAKE), 1000, tau, 5, ctypes.byref(out),
+                                  ctypes.byref(win), ctypes.byref(n)) == m.ERR_INVALID_ARG
+
+
+def test_window_step_checks_before_launch(m):
+    blk = _blocks(m, [128, 128], 128)
+    c = _cache(m, capacity=100)
+    args = lambda flags, queue=None, noise=None, rows=0: m._lib.dp_window_step(
+        ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), 256, ctypes.byref(blk), ctypes.byref(c),
+        ctypes.c_void_p(FAKE + (64 << 20)), None, ctypes.c_void_p(FAKE + (32 << 20)), 2, 64, flags,
+        ctypes.byref(queue) if queue is not None else None, ctypes.c_void_p(noise) if noise else None, rows, 1, None)
+    assert args(m.STEP_POP) == m.ERR_CAPACITY           # head block (128 rows) > cache capacity
+    assert c.n_advances == 0
+    c = _cache(m, capacity=128)
+    assert args(0, noise=FAKE, rows=64) == m.ERR_INVALID_ARG        # push without a queue
+    q = _queue(m, n_slots=2, slot_rows=128, count=2, rows=(128, 128))
+    assert args(0, queue=q, noise=FAKE, rows=128) == m.ERR_CAPACITY  # full queue, no pop
+    assert args(m.STEP_POP, queue=_queue(m, count=0)) == m.ERR_EMPTY

@@ -1,0 +1,222 @@
+"""GPU parity: every kernel of the window step against the CPU oracle on seeded inputs,
+through the C ABI (the Python binding marshals arguments only)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.gpu_util import assert_close, bytes_equal, errors, sample_rows
+from workloads import make_step_inputs, step_config, to_dtype
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+def _table(D, seed=5, T=1000):
+    g = torch.Generator().manual_seed(seed)
+    return torch.tanh(torch.randn(T, 3, D, generator=g)).contiguous()
+
+
+def _randn(shape, seed, dtype, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return to_dtype(torch.randn(*shape, generator=g) * std, dtype)
+
+
+# --------------------------------------------------------------------------- A1 modulation
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rows", [[300, 450, 250], [1], [0, 7, 129, 0]])
+def test_modulate_matches_oracle_bitwise(dp, dtype, rows):
+    D = 1536
+    n = sum(rows)
+    x = _randn((n, D), 1, dtype)
+    table = _table(D)
+    ts = [int(t) for t in np.linspace(0, 999, len(rows)).round()]
+    xd, td = x.cuda(), table.cuda()
+    y = torch.empty_like(xd)
+    blk = dp.blocks_from_table(td, ts, rows)
+    dp.adaln_modulate(xd, y, blk)
+    ro = blk.offsets
+    mod = O.lookup(table, ts)
+    want = O.modulate_rounded(x, ro, mod, dtype)
+    got = y.cpu().double().numpy()
+    assert np.array_equal(got, want), f"mismatches: {int((got != want).sum())}"
+    assert_close(got, O.modulate(x, ro, mod), dtype, "modulate vs fp64")
+    # in place gives the same bytes
+    dp.adaln_modulate(xd, xd, blk)
+    assert bytes_equal(xd, y)
+
+
+# --------------------------------------------------------------------------- A2 attention
+
+ATTN_CASES = [
+    # (H, hd, block rows, cache_len, cache capacity, residual, flags)
+    (2, 64, [500, 300, 200], 300, 333, False, 3),
+    (2, 128, [400, 377], 0, 16, True, 3),
+    (3, 64, [129], 1, 8, False, 3),
+    (1, 64, [1], 0, 1, False, 3),
+    (2, 128, [256, 256], 128, 128, True, 0),
+    (4, 64, [100, 0, 156, 1], 200, 256, True, 1),
+    (2, 64, [5000], 2500, 2500, False, 2),
+]
+
+
+@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"H{c[0]}_hd{c[1]}_n{sum(c[2])}_c{c[3]}")
+def test_attention_bf16_matches_oracle(dp, case):
+    H, hd, rows, Lc, cap, with_res, flags = case
+    D = H * hd
+    n = sum(rows)
+    q, k, v = (_randn((n, D), s, "bf16") for s in (11, 12, 13))
+    ck, cv = (_randn((cap, D), s, "bf16") for s in (14, 15))
+    res = _randn((n, D), 16, "bf16") if with_res else None
+    table = _table(D)
+    ts = [int(t) for t in np.linspace(0, 999, len(rows)).round()]
+    blk = dp.blocks_from_table(table.cuda(), ts, rows)
+    out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
+    dp.window_attention(q.cuda(), k.cuda(), v.cuda(), ck.cuda(), cv.cuda(), Lc, out, H, hd, blk, flags=flags,
+                        residual=res.cuda() if res is not None else None)
+    dp.device_status()
+    want = O.window_attention(q, k, v, ck, cv, Lc, blk.offsets, O.lookup(table, ts), H, hd,
+                              mod_q=bool(flags & 1), gate_out=bool(flags & 2), residual=res)
+    assert_close(out.cpu().double().numpy(), want, "bf16", f"attention {case}")
+
+
+def test_attention_bf16_deterministic(dp):
+    H, hd, n, Lc = 4, 64, 1000, 300
+    D = H * hd
+    q, k, v, ck, cv = (_randn((n, D), s, "bf16").cuda() for s in range(5))
+    blk = dp.blocks_from_table(_table(D).cuda(), [0, 500], [600, 400])
+    a = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
+    b = torch.empty_like(a)
+    dp.window_attention(q, k, v, ck, cv, Lc, a, H, hd, blk)
+    dp.window_attention(q, k, v, ck, cv, Lc, b, H, hd, blk)
+    assert bytes_equal(a, b)
+
+
+@pytest.mark.parametrize("hd", [64, 16])
+def test_attention_f32_matches_oracle(dp, hd):
+    H = 2
+    D = H * hd
+    rows = [100, 90]
+    n = sum(rows)
+    q, k, v = (_randn((n, D), s, "f32") for s in (21, 22, 23))
+    ck, cv = (_randn((70, D), s, "f32") for s in (24, 25))
+    res = _randn((n, D), 26, "f32")
+    table = _table(D)
+    blk = dp.blocks_from_table(table.cuda(), [500, 999], rows)
+    out = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    dp.window_attention(q.cuda(), k.cuda(), v.cuda(), ck.cuda(), cv.cuda(), 70, out, H, hd, blk,
+                        residual=res.cuda())
+    want = O.window_attention(q, k, v, ck, cv, 70, blk.offsets, O.lookup(table, [500, 999]), H, hd, residual=res)
+    assert_close(out.cpu().double().numpy(), want, "f32", "f32 attention")
+
+
+# --------------------------------------------------------------------------- A3 advance
+
+def test_kvcache_advance_bitexact_ring(dp):
+    D, cap = 256, 96
+    c = dp.KVCache(cap, D, dtype=torch.bfloat16, n_slots=3)
+    ref = O.KVCacheRing(3, cap, D)
+    for a, n in enumerate([96, 50, 96, 1, 0, 96, 33]):
+        ke, ve = _randn((max(n, 1), D), 100 + a, "bf16"), _randn((max(n, 1), D), 200 + a, "bf16")
+        dp.kvcache_advance(c, ke.cuda(), ve.cuda(), n)
+        slot = ref.advance(ke, ve, n)
+        assert c.n_advances == a + 1 and c.read_slot() == slot and c.length == n
+        torch.cuda.synchronize()
+        assert np.array_equal(c.k[slot, :n].cpu().double().numpy(), ref.k[slot, :n])
+        assert np.array_equal(c.v[slot, :n].cpu().double().numpy(), ref.v[slot, :n])
+    with pytest.raises(dp.DpError):
+        dp.kvcache_advance(c, ke.cuda(), ve.cuda(), cap + 1)
+
+
+def test_queue_push_pop_mirrored_window(dp):
+    D, slot = 128, 64
+    qu = dp.Queue(3, slot, D, dtype=torch.bfloat16)
+    ref = O.FifoQueue(3)
+    blocks = [_randn((slot, D), 300 + i, "bf16") for i in range(7)] + [_randn((40, D), 399, "bf16")]
+    pushed = 0
+    for i, blk in enumerate(blocks):
+        if qu.count == 3:
+            dp.queue_pop(qu)
+            ref.pop()
+        dp.queue_push(qu, blk.cuda())
+        ref.push(blk)
+        pushed += 1
+        torch.cuda.synchronize()
+        assert qu.rows() == [b.latent.shape[0] for b in ref.blocks]
+        assert np.array_equal(qu.window().cpu().double().numpy(), ref.window())
+    with pytest.raises(dp.DpError):   # nothing may follow the short final block
+        dp.queue_pop(qu)
+        dp.queue_push(qu, blocks[0].cuda())
+
+
+# --------------------------------------------------------------------------- A4 window step
+
+def test_window_step_tiny_f32_two_steps(dp):
+    """tiny_f32: one step with the preset cache, one advance, then a second step that must
+    use the new cache (the exited head block's k')."""
+    cfg = step_config("tiny_f32")
+    x = make_step_inputs(cfg)
+    H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
+    table = x["table"].cuda()
+    blk = dp.blocks_from_table(table, x["timesteps"], cfg.block_rows)
+    ck = x["cache_k"].cuda().view(1, cfg.cache_capacity, D).clone()
+    cv = x["cache_v"].cuda().view(1, cfg.cache_capacity, D).clone()
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.float32, k=ck, v=cv, length=cfg.cache_len)
+    qu = dp.Queue(2, 128, D, dtype=torch.float32)
+    for b in range(2):
+        dp.queue_push(qu, x["noise"].cuda())
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    kv = torch.empty(2, n, D, dtype=torch.float32, device="cuda")
+    out = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    dp.window_step(q, k, v, blk, cache, kv, out, H, hd, pop=True, queue=qu, push_noise=x["noise"].cuda())
+    dp.device_status()
+    mod = O.lookup(x["table"], x["timesteps"])
+    want, kp, vp = O.window_step(x["q"], x["k"], x["v"], x["cache_k"], x["cache_v"], cfg.cache_len, cfg.row_offset,
+                                 mod, H, hd)
+    assert_close(out.cpu().double().numpy(), want, "f32", "step 1")
+    # advance: the cache now holds the head block's k'/v' (bit-exact vs the rounded oracle)
+    n0 = cfg.block_rows[0]
+    kr = O.modulate_rounded(x["k"], cfg.row_offset, mod, "f32")
+    vr = O.modulate_rounded(x["v"], cfg.row_offset, mod, "f32")
+    assert cache.length == n0 and cache.n_advances == 1
+    assert np.array_equal(cache.k[0, :n0].cpu().double().numpy(), kr[:n0])
+    assert np.array_equal(cache.v[0, :n0].cpu().double().numpy(), vr[:n0])
+    assert bytes_equal(cache.k[0, :n0], kv[0, :n0])
+    assert qu.count == 2 and qu.evals() == [1, 0]
+    # step 2 attends to the new cache
+    out2 = torch.empty_like(out)
+    dp.window_step(q, k, v, blk, cache, kv, out2, H, hd)
+    want2, _, _ = O.window_step(x["q"], x["k"], x["v"], kr, vr, n0, cfg.row_offset, mod, H, hd)
+    assert_close(out2.cpu().double().numpy(), want2, "f32", "step 2")
+    assert errors(out2.cpu().double().numpy(), want)[0] > 1e-3   # the cache did change the result
+
+
+@pytest.mark.parametrize("name", ["cogvideo_bf16", "wan_bf16"])
+def test_window_step_full_size_sampled(dp, name):
+    """Full-size bf16 step in the launch configuration the benchmark times; the oracle
+    computes sampled rows (block boundaries, first/last, ragged tail, random)."""
+    cfg = step_config(name)
+    x = make_step_inputs(cfg)
+    H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
+    blk = dp.blocks_from_table(x["table"].cuda(), x["timesteps"], cfg.block_rows)
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.bfloat16, k=x["cache_k"].cuda().view(1, -1, D),
+                       v=x["cache_v"].cuda().view(1, -1, D), length=cfg.cache_len)
+    qu = dp.Queue(cfg.n_blocks, cfg.block_rows[0], D)
+    for _ in range(cfg.n_blocks):
+        dp.queue_push(qu, x["noise"].cuda())
+    kv = torch.empty(2, n, D, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
+    dp.window_step(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), blk, cache, kv, out, H, hd, pop=True, queue=qu,
+                   push_noise=x["noise"].cuda())
+    dp.device_status()
+    rows = sample_rows(cfg.row_offset, n_extra=64)
+    mod = O.lookup(x["table"], x["timesteps"])
+    want, _, _ = O.window_step(x["q"], x["k"], x["v"], x["cache_k"], x["cache_v"], cfg.cache_len, cfg.row_offset,
+                               mod, H, hd, rows=rows)
+    got = out[rows].cpu().double().numpy()
+    assert_close(got, want, "bf16", name)
+    n0 = cfg.block_rows[0]
+    assert bytes_equal(cache.k[0, :n0], kv[0, :n0]) and bytes_equal(cache.v[0, :n0], kv[1, :n0])
+    kr = O.modulate_rounded(x["k"][:n0], [0, n0], mod[:1], "bf16")
+    assert np.array_equal(cache.k[0, :n0].cpu().double().numpy(), kr)
