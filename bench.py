@@ -1,0 +1,376 @@
+"""Window-step benchmark: tokens/s of the DualParal window step and attention TFLOP/s.
+
+One step = the whole hot path on one window: per-block adaLN lookup (host), K/V
+modulation prepass, tensor-core window attention over [cache ; window] with the fused Q
+prologue and gate epilogue, and the queue/cache advance (head block -> cache, fresh noise
+block pushed).  Default workload: the CogVideoX-like window (4 blocks x 2700 tokens,
+2700-token cache, 48 x 64 heads, bf16).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU; every rank runs an
+independent replica (the step needs no exchange between GPUs), the timed region is
+bracketed by barriers and synchronizes, and the slowest rank's time sets the value.
+--impl reference times the CPU oracle (float64 NumPy) on a bounded sample of the same
+workload.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload(name: str):
+    from workloads import step_config
+    if name.startswith("sweep_"):
+        parts = name.split("_")
+        return step_config("sweep", int(parts[1]), ragged=len(parts) > 2 and parts[2] == "ragged")
+    return step_config(name)
+
+
+def describe(cfg) -> str:
+    return (f"{cfg.name}: {cfg.n_blocks} blocks x {cfg.block_rows[0]} tokens (window {cfg.n_win}), "
+            f"cache {cfg.cache_len}, {cfg.n_heads}x{cfg.head_dim} heads, {cfg.dtype}")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = os.path.join("/tmp", f"dp_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.out, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.out) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == len(self.FIELDS):
+                    rows.append(parts)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, nme in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(nme)
+        load = [s for s in sm if s > 0]
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def gpu_arm(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import long_video_diffusion_b200 as dp
+    from workloads import make_step_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workload(args.config)
+    if cfg.dtype != "bf16":
+        raise SystemExit("bench workloads are bf16")
+    x = make_step_inputs(cfg)
+    H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
+    eb = 2
+    table = x["table"].to(dev)
+    blk = dp.blocks_from_table(table, x["timesteps"], cfg.block_rows)
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    noise = x["noise"].to(dev)
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.bfloat16, k=x["cache_k"].to(dev).view(1, -1, D).clone(),
+                       v=x["cache_v"].to(dev).view(1, -1, D).clone(), length=cfg.cache_len)
+    slot_rows = max(cfg.block_rows)
+    queue = dp.Queue(cfg.n_blocks, slot_rows, D, device=dev)
+    for _ in range(cfg.n_blocks):
+        dp.queue_push(queue, noise)
+    kv = torch.empty(2, n, D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(n, D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dp.window_step(q, k, v, blk, cache, kv, out, H, hd, pop=True, queue=queue, push_noise=noise)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dp.device_status()
+
+    # ---- timed region: K window steps, attention timed live by the step's stage events
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(_smi_index(local_rank)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for i in range(args.steps):
+        dp.set_step_events(before_attention=ev_a[i], after_attention=ev_b[i])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dp.set_step_events()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    dp.device_status()
+    ms = t0.elapsed_time(t1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / args.steps
+
+    # ---- e2e: the same step through the public API with pinned host buffers
+    hq, hk, hv = (x[key].pin_memory() for key in ("q", "k", "v"))
+    hnoise = x["noise"].pin_memory()
+    hout = torch.empty(n, D, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dnoise = torch.empty_like(noise)
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dnoise.copy_(hnoise, non_blocking=True)
+        dp.window_step(dq, dk, dv, blk, cache, kv, out, H, hd, pop=True, queue=queue, push_noise=dnoise)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    dp.device_status()
+
+    # slowest rank sets the time
+    vals = torch.tensor([ms, e2e_ms, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, attn_ms = [float(t) for t in vals.tolist()]
+    return cfg, dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, clocks=clocks,
+                     h2d=(hq.numel() + hk.numel() + hv.numel() + hnoise.numel()) * eb, d2h=hout.numel() * eb)
+
+
+def _smi_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [s.strip() for s in vis.split(",") if s.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_step(cfg, x, n_rows: int, head: int, seed: int):
+    """One oracle window step on a bounded sample: head `head` only (heads are independent:
+    its K/V modulation over all window rows, its attention for n_rows random query rows over
+    all keys).  Returns (seconds, seconds extrapolated to the whole step: attention scaled
+    linearly to all rows, everything scaled by the head count)."""
+    import numpy as np
+
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(cfg.n_win, size=min(n_rows, cfg.n_win), replace=False))
+    c0, c1 = head * cfg.head_dim, (head + 1) * cfg.head_dim
+    sl = lambda t: t[:, c0:c1].contiguous()
+    mod = O.lookup(x["table"][:, :, c0:c1].contiguous(), x["timesteps"])
+    q, k, v, ck, cv = sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["cache_k"]), sl(x["cache_v"])
+    t0 = time.perf_counter()
+    kp = O.modulate(k, cfg.row_offset, mod)
+    vp = O.modulate(v, cfg.row_offset, mod)
+    t1 = time.perf_counter()
+    O.window_attention(q, kp, vp, ck, cv, cfg.cache_len, cfg.row_offset, mod, 1, cfg.head_dim, rows=rows)
+    t2 = time.perf_counter()
+    full = ((t1 - t0) + (t2 - t1) * cfg.n_win / len(rows)) * cfg.n_heads
+    return t2 - t0, full, len(rows)
+
+
+def _sample_text(cfg, n_rows):
+    return (f"one head of {cfg.n_heads} per oracle step (heads are independent): its K/V modulation over all "
+            f"{cfg.n_win} window rows and its attention for {n_rows} random query rows over all "
+            f"{cfg.cache_len + cfg.n_win} keys; attention time scaled linearly to all rows, the step's time "
+            f"scaled by the head count")
+
+
+def cpu_baseline(cfg, budget_s: float = 12.0):
+    from workloads import make_step_inputs
+    x = make_step_inputs(cfg)
+    spent, fulls, i = 0.0, [], 0
+    n_rows = 64
+    while (spent < budget_s or i < 3) and i < 4 * cfg.n_heads:
+        s, full, _ = oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=i)
+        spent += s
+        fulls.append(full)
+        i += 1
+    t = statistics.median(fulls)
+    return {"value": cfg.n_win / t, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{i} oracle steps; " + _sample_text(cfg, n_rows) + f"; {spent:.1f} s of CPU work"}
+
+
+def reference_arm(args):
+    """The oracle as the reference arm: W untimed + K timed bounded-sample steps."""
+    from workloads import make_step_inputs
+    cfg = workload(args.config)
+    x = make_step_inputs(cfg)
+    n_rows = 16
+    for i in range(args.warmup):
+        oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=1000 + i)
+    fulls = []
+    for i in range(args.steps):
+        _, full, _ = oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=i)
+        fulls.append(full)
+    ms = 1e3 * statistics.mean(fulls)
+    value = cfg.n_win / (ms / 1e3)
+    cores = _blas_threads()
+    sample = "each step: " + _sample_text(cfg, n_rows)
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(cfg)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="cogvideo_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        cfg, r = gpu_arm(args, rank, world, local_rank)
+    finally:
+        pass
+    if rank == 0:
+        peaks = load_peaks()
+        flop = cfg.attn_flop()
+        ms_step = r["ms"] / args.steps
+        value = world * cfg.n_win * args.steps / (r["ms"] / 1e3)
+        achieved = flop / (r["attn_ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        e2e_ms_step = r["e2e_ms"] / r["e2e_steps"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": describe(cfg), "parallelism": f"replicas x{world} (no exchange)",
+                       "l2": f"inputs larger than L2 (q, k, v {3 * cfg.n_win * cfg.hidden * 2 / 2**20:.0f} MiB "
+                             f"> {L2_BYTES / 2**20:.0f} MiB)"},
+            "attn_tflops": achieved, "attn_ms": r["attn_ms"],
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "attn_bf16_kernel",
+                         "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                         "algorithmic_flop_per_launch": flop},
+            "clocks": r["clocks"],
+            "e2e": {"value": world * cfg.n_win / (e2e_ms_step / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": 3 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -207,6 +207,21 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
                          uint32_t flags, dp_queue* queue, const void* push_noise,
                          int64_t push_rows, dp_dtype dt, void* stream);
 
+/* ---------------------------------------------------------------- profiling */
+
+/* CUDA events (cudaEvent_t handles, caller-created; NULL entries are skipped) that
+ * dp_window_step records on its stream at its stage boundaries, so a caller can time each
+ * kernel inside a running sequence of steps.  The setting is per calling thread and stays
+ * until replaced; dp_set_step_events(NULL) clears it. */
+typedef struct {
+  void* before_modulate;
+  void* before_attention;
+  void* after_attention;
+  void* after_advance;
+} dp_step_events;
+
+dp_status dp_set_step_events(const dp_step_events* ev);
+
 /* ---------------------------------------------------------------- status */
 
 /* Make device `ordinal` current for this thread's later calls. */

@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of the window step runs in the library's CUDA
 kernels, and there is no fallback.  Importing fails loudly when the library has not been
-built (``python -m long_video_diffusion_b200._build``).  PyTorch supplies device memory,
+built (``python long_video_diffusion_b200/_build.py``).  PyTorch supplies device memory,
 streams and the current device; tensors are passed as raw pointers.
 
 The calls mirror include/dp.h:
@@ -33,7 +33,7 @@ MOD_Q, GATE_OUT = 1, 2
 STEP_POP = 1
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_video_diffusion_b200._build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python long_video_diffusion_b200/_build.py` "
                       "(nvcc, sm_100a). There is no non-CUDA implementation.")
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -62,6 +62,11 @@ class DpQueue(ctypes.Structure):
                 ("n_pushed", ctypes.c_int64), ("n_popped", ctypes.c_int64), ("dtype", ctypes.c_int32)]
 
 
+class DpStepEvents(ctypes.Structure):
+    _fields_ = [("before_modulate", ctypes.c_void_p), ("before_attention", ctypes.c_void_p),
+                ("after_attention", ctypes.c_void_p), ("after_advance", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _U32, _F = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
 _SIGS = {
@@ -77,6 +82,7 @@ _SIGS = {
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
     "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
+    "dp_set_step_events": [ctypes.POINTER(DpStepEvents)],
     "dp_set_device": [_I32],
     "dp_device_status": [_P],
     "dp_status_string": [_I32],
@@ -287,6 +293,17 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
                                _ptr(residual), _ptr(out), n_heads, head_dim, STEP_POP if pop else 0,
                                ctypes.byref(queue.desc) if queue is not None else None, _ptr(push_noise),
                                int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
+
+
+def set_step_events(before_modulate=None, before_attention=None, after_attention=None, after_advance=None):
+    """Have window_step record these torch.cuda.Event objects at its stage boundaries
+    (this thread only); call with no arguments to clear."""
+    evs = [before_modulate, before_attention, after_attention, after_advance]
+    if all(e is None for e in evs):
+        _check(_lib.dp_set_step_events(None), "dp_set_step_events")
+        return
+    d = DpStepEvents(*[ctypes.c_void_p(e.cuda_event) if e is not None else None for e in evs])
+    _check(_lib.dp_set_step_events(ctypes.byref(d)), "dp_set_step_events")
 
 
 def device_status(stream=None) -> int:

@@ -1,6 +1,6 @@
 """Build the in-tree CUDA library (libdp_b200.so) for sm_100a with nvcc.
 
-Usage: python -m long_video_diffusion_b200._build   (or __graft_entry__.build()).
+Usage: python long_video_diffusion_b200/_build.py   (or __graft_entry__.build()).
 The library is linked against the static CUDA runtime; the driver API entry point it
 needs (tensor-map encoding) is looked up at run time, so no libcuda link is required.
 """

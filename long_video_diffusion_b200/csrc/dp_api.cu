@@ -14,6 +14,11 @@
 namespace {
 
 thread_local char g_detail[512] = "";
+thread_local dp_step_events g_events = {nullptr, nullptr, nullptr, nullptr};
+
+cudaError_t record(void* ev, cudaStream_t s) {
+  return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev), s) : cudaSuccess;
+}
 
 dp_status fail(dp_status s, const char* fmt, ...) {
   va_list ap;
@@ -179,6 +184,14 @@ const char* dp_status_string(dp_status s) {
 }
 
 const char* dp_last_error_detail(void) { return g_detail; }
+
+dp_status dp_set_step_events(const dp_step_events* ev) {
+  if (ev)
+    g_events = *ev;
+  else
+    g_events = dp_step_events{nullptr, nullptr, nullptr, nullptr};
+  return DP_OK;
+}
 
 dp_status dp_set_device(int32_t ordinal) {
   cudaError_t e = cudaSetDevice(ordinal);
@@ -413,12 +426,16 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   const dp::BlockTable t = to_table(blk);
   const void* src[2] = {k, v};
   void* dst[2] = {kp, vp};
-  cudaError_t e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, s);
+  cudaError_t e = record(g_events.before_modulate, s);
+  if (e == cudaSuccess) e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, s);
+  if (e == cudaSuccess) e = record(g_events.before_attention, s);
   if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
   // A2: attention with the Q prologue and gate epilogue
   st = run_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, 0.0f, blk,
                      DP_MOD_Q | DP_GATE_OUT, dt, s);
   if (st != DP_OK) return st;
+  e = record(g_events.after_attention, s);
+  if (e != cudaSuccess) return cuda_fail(e, "event record");
   // A3: pop (head block's k'/v' -> cache ring) and push (noise -> latent ring), one launch.
   // Descriptors change only after the launch has been accepted.
   dp::CopySeg segs[dp::kMaxCopySegs];
@@ -440,6 +457,8 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
     e = dp::launch_copy(segs, nseg, s);
     if (e != cudaSuccess) return cuda_fail(e, "advance copy");
   }
+  e = record(g_events.after_advance, s);
+  if (e != cudaSuccess) return cuda_fail(e, "event record");
   if (queue)
     for (int i = 0; i < queue->count; ++i) queue->evals[i] += 1;
   if (pop) {

@@ -108,28 +108,28 @@ def window_attention(q, k, v, cache_k, cache_v, cache_len: int, row_offset: Sequ
         o_i  = sum_j p_ij V_j;  out_i = gate_beta(i) * o_i (+ residual_i)
     ``rows`` restricts the computation to a subset of query rows (returned in that order).
     """
-    q = as_f64(q)
     n_win, D = q.shape
     if D != n_heads * head_dim:
         raise ValueError("hidden != n_heads * head_dim")
-    k = as_f64(k)
-    v = as_f64(v)
-    ck = as_f64(cache_k)[:cache_len]
-    cv = as_f64(cache_v)[:cache_len]
     mod = as_f64(mod)
     beta = row_blocks(row_offset, n_win)
     sel = np.arange(n_win) if rows is None else np.asarray(rows, dtype=np.int64)
-    qs = q[sel]
+    qs = as_f64(q[sel] if rows is not None else q)
     if mod_q:
         qs = qs * (1.0 + mod[beta[sel], 1, :]) + mod[beta[sel], 0, :]
-    K = np.concatenate([ck, k], axis=0)
-    V = np.concatenate([cv, v], axis=0)
+    # keys and values: [cache rows 0..L_c ; window rows], laid out head-major [H, L, hd]
+    K = np.concatenate([as_f64(cache_k[:cache_len]), as_f64(k)], axis=0)
+    V = np.concatenate([as_f64(cache_v[:cache_len]), as_f64(v)], axis=0)
+    L = K.shape[0]
+    Kh_all = np.ascontiguousarray(K.reshape(L, n_heads, head_dim).transpose(1, 0, 2))
+    Vh_all = np.ascontiguousarray(V.reshape(L, n_heads, head_dim).transpose(1, 0, 2))
+    del K, V
     scale = (1.0 / math.sqrt(head_dim)) if softmax_scale is None else float(softmax_scale)
     out = np.empty((sel.size, D), dtype=np.float64)
     for h in range(n_heads):
         c0, c1 = h * head_dim, (h + 1) * head_dim
-        Kh = K[:, c0:c1]
-        Vh = V[:, c0:c1]
+        Kh = Kh_all[h]
+        Vh = Vh_all[h]
         for r0 in range(0, sel.size, q_chunk):
             qh = qs[r0:r0 + q_chunk, c0:c1]
             s = (qh @ Kh.T) * scale                 # pass 1: logits and row max
