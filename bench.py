@@ -146,9 +146,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     dp.device_status()
 
-    # ---- timed region: K window steps, attention timed live by the step's stage events
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # ---- timed region: K window steps; each stage is timed live by the library's events
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(_smi_index(local_rank)) if rank == 0 else None
     if world > 1:
@@ -157,19 +155,19 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     if sampler:
         sampler.start()
         time.sleep(0.3)
+    dp.profile_begin(args.steps)
     t0.record(stream)
-    for i in range(args.steps):
-        dp.set_step_events(before_attention=ev_a[i], after_attention=ev_b[i])
+    for _ in range(args.steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
-    dp.set_step_events()
+    mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()
     dp.device_status()
     ms = t0.elapsed_time(t1)
-    attn_ms = sum(a.elapsed_time(b) for a, b in zip(ev_a, ev_b)) / args.steps
+    attn_ms, mod_ms, adv_ms = attn_ms / n_prof, mod_ms / n_prof, adv_ms / n_prof
 
     # ---- e2e: the same step through the public API with pinned host buffers
     hq, hk, hv = (x[key].pin_memory() for key in ("q", "k", "v"))
@@ -202,12 +200,42 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     dp.device_status()
 
     # slowest rank sets the time
-    vals = torch.tensor([ms, e2e_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, attn_ms = [float(t) for t in vals.tolist()]
-    return cfg, dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, clocks=clocks,
+    ms, e2e_ms, attn_ms, mod_ms, adv_ms = max_over_ranks([ms, e2e_ms, attn_ms, mod_ms, adv_ms], dev)
+    return cfg, dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
+                     clocks=clocks,
                      h2d=(hq.numel() + hk.numel() + hv.numel() + hnoise.numel()) * eb, d2h=hout.numel() * eb)
+
+
+def stage_hbm(cfg, r, peaks):
+    """Achieved HBM bandwidth of the two copy-like stages (algorithmic bytes / event time):
+    modulation reads k, v and writes k', v' (4 N_w D e bytes); the advance copies the head
+    block's k'/v' into the cache (4 n_exit D e) and the noise block into both halves of the
+    mirrored ring (3 n_push D e)."""
+    eb = cfg.elem_bytes
+    mod_b = 4 * cfg.n_win * cfg.hidden * eb
+    adv_b = (4 * cfg.block_rows[0] + 3 * cfg.push_rows) * cfg.hidden * eb
+    out = {}
+    for name, b, ms in (("modulate", mod_b, r["mod_ms"]), ("advance", adv_b, r["adv_ms"])):
+        gbs = b / (ms / 1e3) / 1e9 if ms > 0 else None
+        out[name] = {"bytes": b, "ms": ms, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+                     "frac": (gbs / peaks["hbm_gbs"]) if gbs else None}
+    return out
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor(values, dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world: int, n_win: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own window per step (weak scaling)."""
+    return world * n_win * steps / (max_ms / 1e3)
 
 
 def _smi_index(local_rank: int) -> int:
@@ -342,7 +370,7 @@ def main():
         peaks = load_peaks()
         flop = cfg.attn_flop()
         ms_step = r["ms"] / args.steps
-        value = world * cfg.n_win * args.steps / (r["ms"] / 1e3)
+        value = job_throughput(world, cfg.n_win, args.steps, r["ms"])
         achieved = flop / (r["attn_ms"] / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         e2e_ms_step = r["e2e_ms"] / r["e2e_steps"]
@@ -353,11 +381,13 @@ def main():
             "config": {"workload": describe(cfg), "parallelism": f"replicas x{world} (no exchange)",
                        "l2": f"inputs larger than L2 (q, k, v {3 * cfg.n_win * cfg.hidden * 2 / 2**20:.0f} MiB "
                              f"> {L2_BYTES / 2**20:.0f} MiB)"},
-            "attn_tflops": achieved, "attn_ms": r["attn_ms"],
+            "attn_tflops": achieved,
+            "stage_ms": {"modulate": r["mod_ms"], "attention": r["attn_ms"], "advance": r["adv_ms"]},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None, "kernel": "attn_bf16_kernel",
                          "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
                          "algorithmic_flop_per_launch": flop},
+            "stage_hbm": stage_hbm(cfg, r, peaks),
             "clocks": r["clocks"],
             "e2e": {"value": world * cfg.n_win / (e2e_ms_step / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},

@@ -209,18 +209,16 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
 
 /* ---------------------------------------------------------------- profiling */
 
-/* CUDA events (cudaEvent_t handles, caller-created; NULL entries are skipped) that
- * dp_window_step records on its stream at its stage boundaries, so a caller can time each
- * kernel inside a running sequence of steps.  The setting is per calling thread and stays
- * until replaced; dp_set_step_events(NULL) clears it. */
-typedef struct {
-  void* before_modulate;
-  void* before_attention;
-  void* after_attention;
-  void* after_advance;
-} dp_step_events;
-
-dp_status dp_set_step_events(const dp_step_events* ev);
+/* Stage timing of dp_window_step.  After dp_profile_begin(max_steps), the next max_steps
+ * dp_window_step calls on this thread record CUDA events (created and owned by the
+ * library; no device memory) on their stream at the boundaries of the modulation prepass,
+ * the attention and the advance.  dp_profile_end synchronizes on the last recorded event,
+ * returns the summed times in milliseconds (any output pointer may be NULL) and the number
+ * of steps recorded, and releases the events.  INVALID_ARG if max_steps < 1 or if
+ * profiling is already active (begin) / not active (end). */
+dp_status dp_profile_begin(int32_t max_steps);
+dp_status dp_profile_end(float* ms_modulate, float* ms_attention, float* ms_advance,
+                         int32_t* steps);
 
 /* ---------------------------------------------------------------- status */
 

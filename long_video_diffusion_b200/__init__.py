@@ -62,11 +62,6 @@ class DpQueue(ctypes.Structure):
                 ("n_pushed", ctypes.c_int64), ("n_popped", ctypes.c_int64), ("dtype", ctypes.c_int32)]
 
 
-class DpStepEvents(ctypes.Structure):
-    _fields_ = [("before_modulate", ctypes.c_void_p), ("before_attention", ctypes.c_void_p),
-                ("after_attention", ctypes.c_void_p), ("after_advance", ctypes.c_void_p)]
-
-
 _P = ctypes.c_void_p
 _I32, _I64, _U32, _F = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
 _SIGS = {
@@ -82,7 +77,8 @@ _SIGS = {
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
     "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
-    "dp_set_step_events": [ctypes.POINTER(DpStepEvents)],
+    "dp_profile_begin": [_I32],
+    "dp_profile_end": [ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_I32)],
     "dp_set_device": [_I32],
     "dp_device_status": [_P],
     "dp_status_string": [_I32],
@@ -295,15 +291,18 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
                                int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
 
 
-def set_step_events(before_modulate=None, before_attention=None, after_attention=None, after_advance=None):
-    """Have window_step record these torch.cuda.Event objects at its stage boundaries
-    (this thread only); call with no arguments to clear."""
-    evs = [before_modulate, before_attention, after_attention, after_advance]
-    if all(e is None for e in evs):
-        _check(_lib.dp_set_step_events(None), "dp_set_step_events")
-        return
-    d = DpStepEvents(*[ctypes.c_void_p(e.cuda_event) if e is not None else None for e in evs])
-    _check(_lib.dp_set_step_events(ctypes.byref(d)), "dp_set_step_events")
+def profile_begin(max_steps: int) -> None:
+    """Time the stages of the next max_steps window_step calls on this thread."""
+    _check(_lib.dp_profile_begin(int(max_steps)), "dp_profile_begin")
+
+
+def profile_end():
+    """(ms_modulate, ms_attention, ms_advance, steps): summed stage times since profile_begin."""
+    a, b, c = ctypes.c_float(), ctypes.c_float(), ctypes.c_float()
+    n = ctypes.c_int32()
+    _check(_lib.dp_profile_end(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(n)),
+           "dp_profile_end")
+    return a.value, b.value, c.value, n.value
 
 
 def device_status(stream=None) -> int:
@@ -316,3 +315,38 @@ def device_status(stream=None) -> int:
 
 def loaded_library_path() -> str:
     return LIB_PATH
+
+
+# ------------------------------------------------------------------------- long-video run
+
+def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
+    """Step at which block b enters the queue: floor(b * T / W), so that the window holds W
+    blocks in steady state and block b's exit coincides with block b + W's entry."""
+    return (b * n_timesteps) // window_blocks
+
+
+def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
+             queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
+             on_step=None, stream=None) -> int:
+    """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
+    the tail, pop a clean block at the head; every block is evaluated once per step at its
+    own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
+    noise_blocks: device tensors in entry order.  on_step(step, n_win, popped, pushed) is
+    called after each step is enqueued.  Returns the number of steps."""
+    T = len(tau)
+    n_blocks = len(noise_blocks)
+    queue_push(queue, noise_blocks[0], stream=stream)
+    nxt = 1
+    step = 0
+    while queue.count > 0:
+        blk, win, n = queue_blocks(queue, table, tau)
+        pop = queue.evals()[0] + 1 == T
+        push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1
+        window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,
+                    push_noise=noise_blocks[nxt] if push else None, stream=stream, n_win=n)
+        if on_step is not None:
+            on_step(step, n, pop, nxt if push else None)
+        if push:
+            nxt += 1
+        step += 1
+    return step

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "dp.h"
 #include "dp_internal.h"
@@ -14,11 +15,21 @@
 namespace {
 
 thread_local char g_detail[512] = "";
-thread_local dp_step_events g_events = {nullptr, nullptr, nullptr, nullptr};
+// Stage profiling of dp_window_step (per thread): 4 events per recorded step.
+struct Profile {
+  std::vector<cudaEvent_t> ev;
+  int32_t max_steps = 0;
+  int32_t count = 0;
+  bool active = false;
+};
+thread_local Profile g_prof;
 
-cudaError_t record(void* ev, cudaStream_t s) {
-  return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev), s) : cudaSuccess;
+cudaEvent_t prof_event(int stage) {
+  if (!g_prof.active || g_prof.count >= g_prof.max_steps) return nullptr;
+  return g_prof.ev[4 * g_prof.count + stage];
 }
+
+cudaError_t record(cudaEvent_t ev, cudaStream_t s) { return ev ? cudaEventRecord(ev, s) : cudaSuccess; }
 
 dp_status fail(dp_status s, const char* fmt, ...) {
   va_list ap;
@@ -185,12 +196,47 @@ const char* dp_status_string(dp_status s) {
 
 const char* dp_last_error_detail(void) { return g_detail; }
 
-dp_status dp_set_step_events(const dp_step_events* ev) {
-  if (ev)
-    g_events = *ev;
-  else
-    g_events = dp_step_events{nullptr, nullptr, nullptr, nullptr};
+dp_status dp_profile_begin(int32_t max_steps) {
+  if (max_steps < 1) return fail(DP_ERR_INVALID_ARG, "max_steps %d", max_steps);
+  if (g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling already active");
+  g_prof.ev.assign(static_cast<size_t>(4) * max_steps, nullptr);
+  for (auto& e : g_prof.ev) {
+    cudaError_t r = cudaEventCreate(&e);
+    if (r != cudaSuccess) {
+      for (auto& x : g_prof.ev)
+        if (x) cudaEventDestroy(x);
+      g_prof.ev.clear();
+      return cuda_fail(r, "cudaEventCreate");
+    }
+  }
+  g_prof.max_steps = max_steps;
+  g_prof.count = 0;
+  g_prof.active = true;
   return DP_OK;
+}
+
+dp_status dp_profile_end(float* ms_modulate, float* ms_attention, float* ms_advance, int32_t* steps) {
+  if (!g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling not active");
+  double sum[3] = {0.0, 0.0, 0.0};
+  dp_status st = DP_OK;
+  if (g_prof.count > 0) {
+    cudaError_t r = cudaEventSynchronize(g_prof.ev[4 * (g_prof.count - 1) + 3]);
+    for (int i = 0; r == cudaSuccess && i < g_prof.count; ++i)
+      for (int k = 0; r == cudaSuccess && k < 3; ++k) {
+        float ms = 0.0f;
+        r = cudaEventElapsedTime(&ms, g_prof.ev[4 * i + k], g_prof.ev[4 * i + k + 1]);
+        sum[k] += ms;
+      }
+    if (r != cudaSuccess) st = cuda_fail(r, "event timing");
+  }
+  for (auto& e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.active = false;
+  if (ms_modulate) *ms_modulate = static_cast<float>(sum[0]);
+  if (ms_attention) *ms_attention = static_cast<float>(sum[1]);
+  if (ms_advance) *ms_advance = static_cast<float>(sum[2]);
+  if (steps) *steps = g_prof.count;
+  return st;
 }
 
 dp_status dp_set_device(int32_t ordinal) {
@@ -426,15 +472,16 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   const dp::BlockTable t = to_table(blk);
   const void* src[2] = {k, v};
   void* dst[2] = {kp, vp};
-  cudaError_t e = record(g_events.before_modulate, s);
+  cudaEvent_t ev0 = prof_event(0), ev1 = prof_event(1), ev2 = prof_event(2), ev3 = prof_event(3);
+  cudaError_t e = record(ev0, s);
   if (e == cudaSuccess) e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, s);
-  if (e == cudaSuccess) e = record(g_events.before_attention, s);
+  if (e == cudaSuccess) e = record(ev1, s);
   if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
   // A2: attention with the Q prologue and gate epilogue
   st = run_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, 0.0f, blk,
                      DP_MOD_Q | DP_GATE_OUT, dt, s);
   if (st != DP_OK) return st;
-  e = record(g_events.after_attention, s);
+  e = record(ev2, s);
   if (e != cudaSuccess) return cuda_fail(e, "event record");
   // A3: pop (head block's k'/v' -> cache ring) and push (noise -> latent ring), one launch.
   // Descriptors change only after the launch has been accepted.
@@ -457,8 +504,9 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
     e = dp::launch_copy(segs, nseg, s);
     if (e != cudaSuccess) return cuda_fail(e, "advance copy");
   }
-  e = record(g_events.after_advance, s);
+  e = record(ev3, s);
   if (e != cudaSuccess) return cuda_fail(e, "event record");
+  if (ev3) g_prof.count += 1;
   if (queue)
     for (int i = 0; i < queue->count; ++i) queue->evals[i] += 1;
   if (pop) {
