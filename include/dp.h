@@ -20,8 +20,11 @@
  *  - Token tensors are row-major [rows][hidden], hidden = n_heads * head_dim, channel
  *    c = h * head_dim + d.  Window rows are ordered head block (cleanest, smallest
  *    timestep) first.
- *  - Element type is given by dp_dtype: DP_BF16 (bfloat16) or DP_F32 (float).  adaLN
- *    vectors are always float.
+ *  - Element types (dp_dtype): window inputs q, k, v, residual, out, noise and the latent
+ *    queue are DP_BF16 (or DP_F32 for the fp32 path).  The modulated features k', v' and
+ *    the cache are DP_F16 on the bf16 path (11-bit significand: with bf16 features the
+ *    rounding of q', k', v' alone exceeds 2e-2 absolute on peaked softmaxes; f16 features
+ *    saturate at +-65504) and DP_F32 on the fp32 path.  adaLN vectors are always float.
  *  - Ownership: the caller owns every device buffer; the library allocates no device
  *    memory on any call.  Descriptor structs are host-side plain data; the library
  *    updates their counters deterministically.
@@ -56,7 +59,7 @@ typedef enum {
   DP_ERR_EMPTY = -6         /* pop from an empty queue */
 } dp_status;
 
-typedef enum { DP_F32 = 0, DP_BF16 = 1 } dp_dtype;
+typedef enum { DP_F32 = 0, DP_BF16 = 1, DP_F16 = 2 } dp_dtype;
 
 /* dp_window_attention flags */
 #define DP_MOD_Q 1u     /* prologue: q' = q * (1 + scale_b) + shift_b, b = block of the row */
@@ -145,11 +148,13 @@ dp_status dp_queue_blocks(const dp_queue* q, const float* table, int32_t table_r
 /* ---------------------------------------------------------------- A1: modulation */
 
 /* y[i, c] = x[i, c] * (1 + scale_b[c]) + shift_b[c] for every row i of block b, in fp32
- * (one fused multiply-add, 1 + scale rounded to float), rounded to the element type.
- * x, y: DEVICE [n_rows][hidden]; y may equal x (in place), no other overlap.
- * n_rows must equal blk->row_offset[blk->n_blocks]. */
+ * (one fused multiply-add, 1 + scale rounded to float), rounded once to y's type (round to
+ * nearest even; f16 saturates at +-65504).  x: DEVICE [n_rows][hidden] of x_dt; y: DEVICE
+ * [n_rows][hidden] of y_dt; (x_dt, y_dt) is (bf16, bf16), (bf16, f16), (f16, f16) or
+ * (f32, f32), else UNSUPPORTED.  y may equal x when the types match (in place), no other
+ * overlap.  n_rows must equal blk->row_offset[blk->n_blocks]. */
 dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blocks* blk,
-                            dp_dtype dt, void* stream);
+                            dp_dtype x_dt, dp_dtype y_dt, void* stream);
 
 /* ---------------------------------------------------------------- A2: attention */
 
@@ -159,16 +164,18 @@ dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blo
  *   o_i,h = sum_j softmax_j(q'_i,h . K_j,h * softmax_scale) V_j,h,
  *           j over cache rows [0, cache_len) then window rows [0, n_win)
  *   out_i = (DP_GATE_OUT ? gate_b * o_i : o_i) + (residual ? residual_i : 0)
- * q, k, v, residual, out: DEVICE [n_win][hidden]; k and v enter as given (the window's
- * modulated features).  cache_k, cache_v: DEVICE, at least cache_len rows.  residual may
- * be NULL.  out must not overlap any input.  softmax_scale <= 0 selects 1/sqrt(head_dim).
- * bf16: head_dim 64 or 128 (tensor cores, fp32 accumulation and softmax); f32: head_dim
- * a multiple of 4 up to 128 (CUDA cores, full fp32).  UNSUPPORTED otherwise. */
+ * q, residual, out: DEVICE [n_win][hidden] of dt; k, v: DEVICE [n_win][hidden] of
+ * feat_dt, entering as given (the window's modulated features); cache_k, cache_v: DEVICE
+ * feat_dt, at least cache_len rows.  residual may be NULL.  out must not overlap any
+ * input.  softmax_scale <= 0 selects 1/sqrt(head_dim).  (dt, feat_dt) = (bf16, f16) or
+ * (bf16, bf16): tensor cores, head_dim 64 or 128, q' and P rounded to feat_dt, fp32
+ * accumulation and softmax; (f32, f32): CUDA cores, full fp32, head_dim 4, 8, 16, 32, 64
+ * or 128.  UNSUPPORTED otherwise. */
 dp_status dp_window_attention(const void* q, const void* k, const void* v, int64_t n_win,
                               const void* cache_k, const void* cache_v, int64_t cache_len,
                               const void* residual, void* out, int32_t n_heads,
                               int32_t head_dim, float softmax_scale, const dp_blocks* blk,
-                              uint32_t flags, dp_dtype dt, void* stream);
+                              uint32_t flags, dp_dtype dt, dp_dtype feat_dt, void* stream);
 
 /* ---------------------------------------------------------------- A3: advance */
 
@@ -191,7 +198,7 @@ dp_status dp_queue_pop(dp_queue* q);
 
 /* One window step:
  *   1. k' = modulate(k), v' = modulate(v) into kv_work (DEVICE scratch, caller-allocated,
- *      2 * n_win * hidden elements: k' then v');
+ *      2 * n_win * hidden feature elements: k' at element 0, v' at element n_win * hidden);
  *   2. out = dp_window_attention(q, k', v', cache, DP_MOD_Q | DP_GATE_OUT, residual);
  *   3. queue (if given): every live block's evals += 1;
  *   4. if flags & DP_STEP_POP: the head block (rows [0, row_offset[1])) exits — its k'/v'
@@ -199,8 +206,10 @@ dp_status dp_queue_pop(dp_queue* q);
  *      given) pops its head;
  *   5. if push_noise: it is pushed at the queue's tail (dp_queue_push; needs queue).
  * Steps 4 and 5 run as one copy kernel after the attention on the same stream.  All
- * argument checks (including capacities) happen before anything is enqueued.  q, k and v
- * may alias one another (the queue's window); out and kv_work overlap nothing. */
+ * argument checks (including capacities) happen before anything is enqueued.  q, k, v,
+ * residual, out, push_noise and the queue are of type dt (bf16 or f32); kv_work and the
+ * cache hold features (f16 for bf16, f32 for f32).  q, k and v may alias one another (the
+ * queue's window); out and kv_work overlap nothing. */
 dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_win,
                          const dp_blocks* blk, dp_kvcache* cache, void* kv_work,
                          const void* residual, void* out, int32_t n_heads, int32_t head_dim,

@@ -28,7 +28,7 @@ MAX_BLOCKS = 16
 MAX_SLOTS = 16
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_CAPACITY, ERR_TIMEOUT, ERR_EMPTY = 0, -1, -2, -3, -4, -5, -6
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 MOD_Q, GATE_OUT = 1, 2
 STEP_POP = 1
 
@@ -69,9 +69,9 @@ _SIGS = {
                              ctypes.POINTER(_I32), _I32],
     "dp_queue_blocks": [ctypes.POINTER(DpQueue), _P, _I32, ctypes.POINTER(_I32), _I32,
                         ctypes.POINTER(DpBlocks), ctypes.POINTER(_P), ctypes.POINTER(_I64)],
-    "dp_adaln_modulate": [_P, _P, _I64, ctypes.POINTER(DpBlocks), _I32, _P],
+    "dp_adaln_modulate": [_P, _P, _I64, ctypes.POINTER(DpBlocks), _I32, _I32, _P],
     "dp_window_attention": [_P, _P, _P, _I64, _P, _P, _I64, _P, _P, _I32, _I32, _F,
-                            ctypes.POINTER(DpBlocks), _U32, _I32, _P],
+                            ctypes.POINTER(DpBlocks), _U32, _I32, _I32, _P],
     "dp_kvcache_advance": [ctypes.POINTER(DpKvcache), _P, _P, _I64, _P],
     "dp_queue_push": [ctypes.POINTER(DpQueue), _P, _I64, _P],
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
@@ -113,6 +113,8 @@ def _dtype(t: torch.Tensor) -> int:
         return BF16
     if t.dtype == torch.float32:
         return F32
+    if t.dtype == torch.float16:
+        return F16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -157,10 +159,16 @@ def blocks_from_table(table: torch.Tensor, timesteps: Sequence[int], block_rows:
 
 # ------------------------------------------------------------------------- state
 
+def feature_dtype(window_dtype: torch.dtype) -> torch.dtype:
+    """Element type of the modulated features k', v' and of the cache for a window of
+    ``window_dtype``: f16 for bf16 windows, f32 for f32 windows."""
+    return torch.float32 if window_dtype == torch.float32 else torch.float16
+
+
 class KVCache:
     """The feature-cache ring (device buffers [n_slots, capacity, hidden] owned here)."""
 
-    def __init__(self, capacity: int, hidden: int, dtype=torch.bfloat16, n_slots: int = 1,
+    def __init__(self, capacity: int, hidden: int, dtype=torch.float16, n_slots: int = 1,
                  device="cuda", k: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None,
                  length: int = 0):
         self.k = torch.zeros(n_slots, capacity, hidden, dtype=dtype, device=device) if k is None else k
@@ -243,7 +251,8 @@ def queue_blocks(queue: Queue, table: torch.Tensor, tau: Sequence[int]):
 # ------------------------------------------------------------------------- A1..A4
 
 def adaln_modulate(x: torch.Tensor, y: torch.Tensor, blocks: DpBlocks, stream=None) -> None:
-    _check(_lib.dp_adaln_modulate(_ptr(x), _ptr(y), x.shape[0], ctypes.byref(blocks), _dtype(x),
+    """y = x * (1 + scale_b) + shift_b, rounded to y's dtype (bf16->bf16, bf16->f16, f16->f16, f32->f32)."""
+    _check(_lib.dp_adaln_modulate(_ptr(x), _ptr(y), x.shape[0], ctypes.byref(blocks), _dtype(x), _dtype(y),
                                   _stream(x, stream)), "dp_adaln_modulate")
 
 
@@ -252,7 +261,7 @@ def window_attention(q, k, v, cache_k, cache_v, cache_len: int, out, n_heads: in
                      softmax_scale: float = 0.0, stream=None) -> None:
     _check(_lib.dp_window_attention(_ptr(q), _ptr(k), _ptr(v), q.shape[0], _ptr(cache_k), _ptr(cache_v),
                                     int(cache_len), _ptr(residual), _ptr(out), n_heads, head_dim,
-                                    float(softmax_scale), ctypes.byref(blocks), flags, _dtype(q),
+                                    float(softmax_scale), ctypes.byref(blocks), flags, _dtype(q), _dtype(k),
                                     _stream(q, stream)), "dp_window_attention")
 
 
@@ -275,7 +284,8 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
                 pop: bool = False, queue: Optional[Queue] = None, push_noise=None, push_rows=None,
                 residual=None, stream=None, n_win: Optional[int] = None) -> None:
     """One window step (see dp_window_step).  q, k, v are tensors or raw device addresses
-    (n_win then required), e.g. the queue's live window."""
+    (n_win then required), e.g. the queue's live window.  kv_work holds at least
+    2 * n_win * hidden feature elements (k' first, v' at element n_win * hidden)."""
     if isinstance(q, torch.Tensor):
         ref = q
         n = q.shape[0]

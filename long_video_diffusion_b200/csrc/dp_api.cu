@@ -45,9 +45,17 @@ dp_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int elem_bytes(dp_dtype dt) { return dt == DP_BF16 ? 2 : 4; }
+int elem_bytes(dp_dtype dt) { return dt == DP_F32 ? 4 : 2; }
 
-bool dtype_ok(dp_dtype dt) { return dt == DP_BF16 || dt == DP_F32; }
+bool dtype_ok(dp_dtype dt) { return dt == DP_BF16 || dt == DP_F16 || dt == DP_F32; }
+
+// Element type of the modulated features (k', v', cache) for a window of type dt.
+dp_dtype feature_dtype(dp_dtype dt) { return dt == DP_F32 ? DP_F32 : DP_F16; }
+
+bool modulate_pair_ok(dp_dtype x, dp_dtype y) {
+  return (x == DP_BF16 && (y == DP_BF16 || y == DP_F16)) || (x == DP_F16 && y == DP_F16) ||
+         (x == DP_F32 && y == DP_F32);
+}
 
 // Row pitch must be a whole number of 16-byte vectors.
 bool hidden_ok(int32_t hidden, dp_dtype dt) {
@@ -304,8 +312,11 @@ dp_status dp_queue_blocks(const dp_queue* q, const float* table, int32_t table_r
   return DP_OK;
 }
 
-dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blocks* blk, dp_dtype dt, void* stream) {
-  if (!dtype_ok(dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blocks* blk, dp_dtype x_dt,
+                            dp_dtype y_dt, void* stream) {
+  if (!dtype_ok(x_dt) || !dtype_ok(y_dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+  if (!modulate_pair_ok(x_dt, y_dt)) return fail(DP_ERR_UNSUPPORTED, "modulation %d -> %d", x_dt, y_dt);
+  const dp_dtype dt = x_dt;
   if (!x || !y || !aligned16(x) || !aligned16(y)) return fail(DP_ERR_INVALID_ARG, "x/y NULL or misaligned");
   if (n_rows <= 0) return fail(DP_ERR_INVALID_ARG, "n_rows %lld", static_cast<long long>(n_rows));
   if (!blk) return fail(DP_ERR_INVALID_ARG, "block table is NULL");
@@ -315,7 +326,7 @@ dp_status dp_adaln_modulate(const void* x, void* y, int64_t n_rows, const dp_blo
   const dp::BlockTable t = to_table(blk);
   const void* src[1] = {x};
   void* dst[1] = {y};
-  cudaError_t e = dp::launch_modulate(src, dst, 1, n_rows, blk->hidden, t, dt, static_cast<cudaStream_t>(stream));
+  cudaError_t e = dp::launch_modulate(src, dst, 1, n_rows, blk->hidden, t, x_dt, y_dt, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
   return DP_OK;
 }
@@ -324,8 +335,11 @@ namespace {
 
 dp_status check_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* ck, const void* cv,
                           int64_t cache_len, const void* residual, void* out, int32_t n_heads, int32_t head_dim,
-                          const dp_blocks* blk, dp_dtype dt) {
-  if (!dtype_ok(dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+                          const dp_blocks* blk, dp_dtype dt, dp_dtype ft) {
+  if (!dtype_ok(dt) || !dtype_ok(ft)) return fail(DP_ERR_INVALID_ARG, "dtype");
+  const bool tc = dt == DP_BF16 && (ft == DP_F16 || ft == DP_BF16);
+  if (!tc && !(dt == DP_F32 && ft == DP_F32))
+    return fail(DP_ERR_UNSUPPORTED, "window/feature dtypes %d/%d (bf16/f16, bf16/bf16 or f32/f32)", dt, ft);
   if (!q || !k || !v || !out) return fail(DP_ERR_INVALID_ARG, "q/k/v/out NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (residual && !aligned16(residual)))
     return fail(DP_ERR_INVALID_ARG, "pointer not 16-byte aligned");
@@ -336,7 +350,7 @@ dp_status check_attention(const void* q, const void* k, const void* v, int64_t n
   if (n_heads <= 0 || head_dim <= 0) return fail(DP_ERR_INVALID_ARG, "n_heads/head_dim");
   const int64_t hidden = static_cast<int64_t>(n_heads) * head_dim;
   if (hidden > INT32_MAX || !hidden_ok(static_cast<int32_t>(hidden), dt)) return fail(DP_ERR_INVALID_ARG, "hidden");
-  if (dt == DP_BF16 && head_dim != 64 && head_dim != 128)
+  if (tc && head_dim != 64 && head_dim != 128)
     return fail(DP_ERR_UNSUPPORTED, "bf16 head_dim %d (64 or 128 supported)", head_dim);
   if (dt == DP_F32 && head_dim != 4 && head_dim != 8 && head_dim != 16 && head_dim != 32 && head_dim != 64 &&
       head_dim != 128)
@@ -348,7 +362,8 @@ dp_status check_attention(const void* q, const void* k, const void* v, int64_t n
 
 dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* ck, const void* cv,
                         int64_t cache_len, const void* residual, void* out, int32_t n_heads, int32_t head_dim,
-                        float softmax_scale, const dp_blocks* blk, uint32_t flags, dp_dtype dt, cudaStream_t s) {
+                        float softmax_scale, const dp_blocks* blk, uint32_t flags, dp_dtype dt, dp_dtype ft,
+                        cudaStream_t s) {
   dp::AttnArgs a;
   a.q = q;
   a.k = k;
@@ -367,7 +382,7 @@ dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_w
   a.bt = to_table(blk);
   dp_status st = status_ptr(&a.status);
   if (st != DP_OK) return st;
-  cudaError_t e = dt == DP_BF16 ? dp::launch_attention_bf16(a, s) : dp::launch_attention_f32(a, s);
+  cudaError_t e = dt == DP_BF16 ? dp::launch_attention_tc(a, ft == DP_F16, s) : dp::launch_attention_f32(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return DP_OK;
 }
@@ -377,11 +392,12 @@ dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_w
 dp_status dp_window_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* cache_k,
                               const void* cache_v, int64_t cache_len, const void* residual, void* out,
                               int32_t n_heads, int32_t head_dim, float softmax_scale, const dp_blocks* blk,
-                              uint32_t flags, dp_dtype dt, void* stream) {
-  dp_status st = check_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, blk, dt);
+                              uint32_t flags, dp_dtype dt, dp_dtype feat_dt, void* stream) {
+  dp_status st =
+      check_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, blk, dt, feat_dt);
   if (st != DP_OK) return st;
   return run_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, softmax_scale,
-                       blk, flags, dt, static_cast<cudaStream_t>(stream));
+                       blk, flags, dt, feat_dt, static_cast<cudaStream_t>(stream));
 }
 
 dp_status dp_kvcache_advance(dp_kvcache* c, const void* k_exit, const void* v_exit, int64_t n_exit, void* stream) {
@@ -440,18 +456,22 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   const int64_t hidden64 = static_cast<int64_t>(n_heads) * head_dim;
   if (n_heads <= 0 || head_dim <= 0 || hidden64 > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_heads/head_dim");
   const int32_t hidden = static_cast<int32_t>(hidden64);
-  dp_status st = check_cache(cache, hidden, dt);
+  if (!dtype_ok(dt)) return fail(DP_ERR_INVALID_ARG, "dtype");
+  const dp_dtype ft = feature_dtype(dt);
+  dp_status st = check_cache(cache, hidden, ft);
   if (st != DP_OK) return st;
   if (!kv_work || !aligned16(kv_work)) return fail(DP_ERR_INVALID_ARG, "kv_work NULL or misaligned");
   const int64_t rslot = cache_read_slot(cache);
-  const int64_t row_bytes = hidden64 * elem_bytes(dt);
+  const int64_t row_bytes = hidden64 * elem_bytes(ft);     // features: k', v', cache
+  const int64_t in_row_bytes = hidden64 * elem_bytes(dt);  // window inputs and the latent queue
   const char* ck = static_cast<const char*>(cache->k) + rslot * cache->capacity * row_bytes;
   const char* cv = static_cast<const char*>(cache->v) + rslot * cache->capacity * row_bytes;
   const int64_t cache_len = cache->len[rslot];
   char* kp = static_cast<char*>(kv_work);
   char* vp = kp + n_win * row_bytes;
-  st = check_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, blk, dt);
+  st = check_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, blk, dt, ft);
   if (st != DP_OK) return st;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return fail(DP_ERR_INVALID_ARG, "k/v NULL or misaligned");
   if (out == kv_work) return fail(DP_ERR_INVALID_ARG, "out aliases kv_work");
   const bool pop = (flags & DP_STEP_POP) != 0;
   const int64_t n_exit = blk->row_offset[1];
@@ -474,12 +494,12 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   void* dst[2] = {kp, vp};
   cudaEvent_t ev0 = prof_event(0), ev1 = prof_event(1), ev2 = prof_event(2), ev3 = prof_event(3);
   cudaError_t e = record(ev0, s);
-  if (e == cudaSuccess) e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, s);
+  if (e == cudaSuccess) e = dp::launch_modulate(src, dst, 2, n_win, hidden, t, dt, ft, s);
   if (e == cudaSuccess) e = record(ev1, s);
   if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
   // A2: attention with the Q prologue and gate epilogue
   st = run_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, 0.0f, blk,
-                     DP_MOD_Q | DP_GATE_OUT, dt, s);
+                     DP_MOD_Q | DP_GATE_OUT, dt, ft, s);
   if (st != DP_OK) return st;
   e = record(ev2, s);
   if (e != cudaSuccess) return cuda_fail(e, "event record");
@@ -496,7 +516,7 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
     const int32_t head_after = (queue->head + ((pop && queue) ? 1 : 0)) % queue->n_slots;
     const int32_t count_after = queue->count - (pop ? 1 : 0);
     const int32_t p = (head_after + count_after) % queue->n_slots;
-    const int64_t bytes = push_rows * row_bytes;
+    const int64_t bytes = push_rows * in_row_bytes;
     segs[nseg++] = {push_noise, queue_slot(queue, p), bytes};
     segs[nseg++] = {push_noise, queue_slot(queue, p + queue->n_slots), bytes};
   }

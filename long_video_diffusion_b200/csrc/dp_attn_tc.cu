@@ -7,6 +7,11 @@
 //   o_i  = softmax_j(q'_i . K_j * scale) V_j         (j: cache rows, then window rows)
 //   out_i = gate_b * o_i (+ residual_i)              (epilogue)
 //
+// Operands: the raw window q is bf16; the modulated features q', k', v' and the softmax
+// weights P enter the tensor cores as 16-bit values of one type, f16 by default (11-bit
+// significand: rounding the modulated features to bf16 alone costs about 2.5e-2 absolute on
+// peaked softmaxes, f16 about 3e-3) or bf16; both accumulate in fp32.
+//
 // Design (one CTA = two 128-row query tiles of one head; keys in 128-row tiles):
 //   warps 0-3  softmax warpgroup for query tile 0 (one thread per query row)
 //   warps 4-7  softmax warpgroup for query tile 1
@@ -74,7 +79,7 @@ struct Layout {
 };
 
 struct Params {
-  const __nv_bfloat16* q;
+  const __nv_bfloat16* q;  // raw window queries (bf16)
   const __nv_bfloat16* residual;
   __nv_bfloat16* out;
   int64_t n_win;
@@ -102,9 +107,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
 
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-template <int HD>
+template <int HD, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+    window_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                      const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
                      const Params p) {
   using L = Layout<HD>;
@@ -194,8 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, HD, true);
+      constexpr uint32_t idS = idesc_f32acc(Operand<F16>::kFmt, BM, BN, false);
+      constexpr uint32_t idPV = idesc_f32acc(Operand<F16>::kFmt, BM, HD, true);
       auto issue_s = [&](int g, int st) {
         const uint32_t qa = sb + L::OFF_Q + g * L::Q_BYTES;
         const uint32_t ka = sb + L::OFF_K + st * L::KV_BYTES;
@@ -275,23 +280,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < HD / 8; ++c) {
         uint4 outv = make_uint4(0, 0, 0, 0);
         if (row_ok) {
-          uint4 raw = src[c];
+          const uint4 raw = src[c];
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          float xf[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(x2[e]);
+            xf[2 * e] = f.x;
+            xf[2 * e + 1] = f.y;
+          }
           if (p.flags & DP_MOD_Q) {
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
             const float4 sh0 = ld_f4(shift + c * 8), sh1 = ld_f4(shift + c * 8 + 4);
             const float4 sc0 = ld_f4(scale + c * 8), sc1 = ld_f4(scale + c * 8 + 4);
             const float sh[8] = {sh0.x, sh0.y, sh0.z, sh0.w, sh1.x, sh1.y, sh1.z, sh1.w};
             const float sc[8] = {sc0.x, sc0.y, sc0.z, sc0.w, sc1.x, sc1.y, sc1.z, sc1.w};
-            uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 xf = __bfloat1622float2(x2[e]);
-              o[e] = pack_bf16x2(fmaf(xf.x, 1.0f + sc[2 * e], sh[2 * e]), fmaf(xf.y, 1.0f + sc[2 * e + 1], sh[2 * e + 1]));
-            }
-            outv = make_uint4(o[0], o[1], o[2], o[3]);
-          } else {
-            outv = raw;
+            for (int e = 0; e < 8; ++e) xf[e] = fmaf(xf[e], 1.0f + sc[e], sh[e]);
           }
+          outv = make_uint4(Operand<F16>::pack(xf[0], xf[1]), Operand<F16>::pack(xf[2], xf[3]),
+                            Operand<F16>::pack(xf[4], xf[5]), Operand<F16>::pack(xf[6], xf[7]));
         }
         const int chunk = c >> 3, w = c & 7;
         *reinterpret_cast<uint4*>(sq + chunk * L::CHUNK_BYTES + t * 128 + ((w ^ (t & 7)) << 4)) = outv;
@@ -366,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float a = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c]), p.scale_log2, nm));
           const float b = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c + 1]), p.scale_log2, nm));
           l_sum += a + b;
-          pk[c] = pack_bf16x2(a, b);
+          pk[c] = Operand<F16>::pack(a, b);
         }
         tmem_st16(trow + s_col + i * 16, pk);
       }
@@ -450,15 +457,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-template <int HD>
+template <int HD, bool F16>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   using L = Layout<HD>;
   CUtensorMap tkc, tvc, tkw, tvw;
-  if (!encode_tmap_bf16(&tkw, a.k, a.n_win, a.hidden) || !encode_tmap_bf16(&tvw, a.v, a.n_win, a.hidden))
+  if (!encode_tmap_16(&tkw, a.k, a.n_win, a.hidden, F16) || !encode_tmap_16(&tvw, a.v, a.n_win, a.hidden, F16))
     return cudaErrorInvalidValue;
   if (a.cache_len > 0) {
-    if (!encode_tmap_bf16(&tkc, a.cache_k, a.cache_len, a.hidden) ||
-        !encode_tmap_bf16(&tvc, a.cache_v, a.cache_len, a.hidden))
+    if (!encode_tmap_16(&tkc, a.cache_k, a.cache_len, a.hidden, F16) ||
+        !encode_tmap_16(&tvc, a.cache_v, a.cache_len, a.hidden, F16))
       return cudaErrorInvalidValue;
   } else {
     tkc = tkw;
@@ -481,42 +488,42 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool attr_set[64] = {};
+  static bool attr_set[64] = {};  // per instantiation and device
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(attn_bf16_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    e = cudaFuncSetAttribute(window_attn_tc_kernel<HD, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     // setmaxnreg.inc waits for registers the launch did not provide: refuse to launch if
     // the compiled register count is below the split's assumption.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, attn_bf16_kernel<HD>);
+    e = cudaFuncGetAttributes(&fa, window_attn_tc_kernel<HD, F16>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
     attr_set[dev] = true;
   }
   const int64_t grid = static_cast<int64_t>(p.n_qpairs) * a.n_heads;
-  attn_bf16_kernel<HD><<<static_cast<unsigned>(grid), kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
+  window_attn_tc_kernel<HD, F16><<<static_cast<unsigned>(grid), kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-bool encode_tmap_bf16(void* tmap, const void* base, int64_t rows, int hidden) {
+bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, bool f16) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(hidden) * 2};
   cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(static_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = fn(static_cast<CUtensorMap*>(tmap), f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
-  if (a.head_dim == 64) return launch_hd<64>(a, s);
-  if (a.head_dim == 128) return launch_hd<128>(a, s);
+cudaError_t launch_attention_tc(const AttnArgs& a, bool f16_features, cudaStream_t s) {
+  if (a.head_dim == 64) return f16_features ? launch_hd<64, true>(a, s) : launch_hd<64, false>(a, s);
+  if (a.head_dim == 128) return f16_features ? launch_hd<128, true>(a, s) : launch_hd<128, false>(a, s);
   return cudaErrorInvalidValue;
 }
 

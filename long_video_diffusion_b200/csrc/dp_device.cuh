@@ -220,10 +220,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, dense, no negation.
-// b_mn_major selects an MN-major B operand.  N >> 3 at bit 17, M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+// Instruction descriptor, kind::f16: fp32 accumulator (bit 4), A and B of one 16-bit type
+// (ab_fmt at bits 7 and 10: 0 = f16, 1 = bf16), dense, no negation.  b_mn_major selects an
+// MN-major B operand (bit 16).  N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t ab_fmt, int M, int N, bool b_mn_major) {
+  return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -237,5 +238,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// Round to nearest even into f16, saturating to +-65504 instead of overflowing to inf.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 16-bit tensor-core operand type: F16 = true selects f16 (11-bit significand), else bf16.
+template <bool F16>
+struct Operand {
+  static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor A/B format
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    if constexpr (F16)
+      return pack_f16x2_sat(lo, hi);
+    else
+      return pack_bf16x2(lo, hi);
+  }
+};
 
 }  // namespace dp

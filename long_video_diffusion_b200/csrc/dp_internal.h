@@ -58,14 +58,16 @@ struct CopySeg {
 };
 constexpr int kMaxCopySegs = 4;
 
-cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s);
+// Tensor-core path: q, residual, out bf16; k, v, cache f16 (f16_features) or bf16.
+cudaError_t launch_attention_tc(const AttnArgs& a, bool f16_features, cudaStream_t s);
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s);
+// x_dt -> y_dt: bf16 -> bf16, bf16 -> f16 (saturating), f16 -> f16, f32 -> f32.
 cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, int64_t n_rows,
-                            int hidden, const BlockTable& bt, dp_dtype dt, cudaStream_t s);
+                            int hidden, const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s);
 cudaError_t launch_copy(const CopySeg* segs, int nseg, cudaStream_t s);
 
-// Host-side helper: encode a 2-D bf16 tensor map [rows][hidden] with a {64, 128} box and
-// 128-byte swizzle (defined in dp_attn_bf16.cu).
-bool encode_tmap_bf16(void* tmap, const void* base, int64_t rows, int hidden);
+// Host-side helper: encode a 2-D 16-bit (f16 or bf16) tensor map [rows][hidden] with a
+// {64, 128} box and 128-byte swizzle (defined in dp_attn_tc.cu).
+bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, bool f16);
 
 }  // namespace dp

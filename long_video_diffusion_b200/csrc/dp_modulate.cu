@@ -3,7 +3,7 @@
 // Modulation (each block conditioned on its own timestep: "Minute-Long Videos with Dual
 // Parallelisms", abstract, blocks at progressively decreasing noise levels; pith.science
 // review, Section 3.1): y = x * (1 + scale_b) + shift_b per channel, one fp32 FMA per
-// element, rounded once to the element type.  Each thread moves 16-byte vectors (8 bf16
+// element, rounded once to the output type (f16 saturates at +-65504).  Each thread moves 16-byte vectors (8 bf16
 // or 4 fp32) with four independent vectors in flight; the grid is a multiple of the SM
 // count and strides over all rows of every segment.
 //
@@ -11,8 +11,10 @@
 // block enters the latent ring; review, key machinery and Section 3.2): up to four
 // (src, dst, bytes) segments in one launch, 16-byte vectors, bit-exact.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "dp_device.cuh"
 #include "dp_internal.h"
 
 namespace dp {
@@ -27,38 +29,69 @@ struct ModSegs {
   uint4* dst[2];
 };
 
-__device__ __forceinline__ uint4 mod_vec_bf16(uint4 x, const float* sh, const float* sc) {
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(sh)), s1 = __ldg(reinterpret_cast<const float4*>(sh) + 1);
-  const float4 c0 = __ldg(reinterpret_cast<const float4*>(sc)), c1 = __ldg(reinterpret_cast<const float4*>(sc) + 1);
-  const float shv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  const float scv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-  uint32_t o[4];
+// Element formats of a 16-byte vector: 8 bf16, 8 f16 or 4 fp32.
+enum Fmt { kBF16 = 0, kF16 = 1, kF32 = 2 };
+
+template <int F>
+__device__ __forceinline__ void unpack8(uint4 x, float (&f)[8]) {
+  if constexpr (F == kBF16) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(x2[e]);
-    __nv_bfloat162 r = __floats2bfloat162_rn(fmaf(f.x, 1.0f + scv[2 * e], shv[2 * e]),
-                                             fmaf(f.y, 1.0f + scv[2 * e + 1], shv[2 * e + 1]));
-    o[e] = *reinterpret_cast<uint32_t*>(&r);
+    for (int e = 0; e < 4; ++e) {
+      const float2 t = __bfloat1622float2(h[e]);
+      f[2 * e] = t.x;
+      f[2 * e + 1] = t.y;
+    }
+  } else if constexpr (F == kF16) {
+    const __half2* h = reinterpret_cast<const __half2*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 t = __half22float2(h[e]);
+      f[2 * e] = t.x;
+      f[2 * e + 1] = t.y;
+    }
+  } else {
+    const float4 t = *reinterpret_cast<const float4*>(&x);
+    f[0] = t.x, f[1] = t.y, f[2] = t.z, f[3] = t.w;
   }
-  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ uint4 mod_vec_f32(uint4 x, const float* sh, const float* sc) {
-  const float4 s = __ldg(reinterpret_cast<const float4*>(sh));
-  const float4 c = __ldg(reinterpret_cast<const float4*>(sc));
-  float4 f = *reinterpret_cast<float4*>(&x);
-  f.x = fmaf(f.x, 1.0f + c.x, s.x);
-  f.y = fmaf(f.y, 1.0f + c.y, s.y);
-  f.z = fmaf(f.z, 1.0f + c.z, s.z);
-  f.w = fmaf(f.w, 1.0f + c.w, s.w);
-  return *reinterpret_cast<uint4*>(&f);
+template <int F>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  if constexpr (F == kBF16) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+  } else if constexpr (F == kF16) {
+    return make_uint4(pack_f16x2_sat(f[0], f[1]), pack_f16x2_sat(f[2], f[3]), pack_f16x2_sat(f[4], f[5]),
+                      pack_f16x2_sat(f[6], f[7]));
+  } else {
+    const float4 t = make_float4(f[0], f[1], f[2], f[3]);
+    return *reinterpret_cast<const uint4*>(&t);
+  }
 }
 
-template <bool BF16>
+// y = x * (1 + scale) + shift on one 16-byte vector; 1 + scale formed in fp32, one FMA.
+template <int FI, int FO>
+__device__ __forceinline__ uint4 mod_vec(uint4 x, const float* sh, const float* sc) {
+  constexpr int VE = FI == kF32 ? 4 : 8;
+  float f[8], shv[8], scv[8];
+  unpack8<FI>(x, f);
+#pragma unroll
+  for (int v = 0; v < VE / 4; ++v) {
+    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sh) + v);
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(sc) + v);
+    shv[4 * v] = s4.x, shv[4 * v + 1] = s4.y, shv[4 * v + 2] = s4.z, shv[4 * v + 3] = s4.w;
+    scv[4 * v] = c4.x, scv[4 * v + 1] = c4.y, scv[4 * v + 2] = c4.z, scv[4 * v + 3] = c4.w;
+  }
+#pragma unroll
+  for (int e = 0; e < VE; ++e) f[e] = fmaf(f[e], 1.0f + scv[e], shv[e]);
+  return pack8<FO>(f);
+}
+
+template <int FI, int FO>
 __global__ void __launch_bounds__(kThreads) modulate_kernel(ModSegs segs, uint32_t vec_per_row, uint32_t vec_per_seg,
                                                             int hidden, BlockTable bt) {
-  constexpr int VE = BF16 ? 8 : 4;  // elements per 16-byte vector
+  constexpr int VE = FI == kF32 ? 4 : 8;  // elements per 16-byte vector
   const uint4* src = segs.src[blockIdx.y];
   uint4* dst = segs.dst[blockIdx.y];
   const uint32_t stride = gridDim.x * kThreads;
@@ -76,8 +109,7 @@ __global__ void __launch_bounds__(kThreads) modulate_kernel(ModSegs segs, uint32
       const uint32_t row = idx[u] / vec_per_row;
       const uint32_t col = (idx[u] - row * vec_per_row) * VE;
       const float* m = block_mod(bt, block_of_row(bt, row));
-      const uint4 y = BF16 ? mod_vec_bf16(x[u], m + col, m + hidden + col) : mod_vec_f32(x[u], m + col, m + hidden + col);
-      dst[idx[u]] = y;
+      dst[idx[u]] = mod_vec<FI, FO>(x[u], m + col, m + hidden + col);
     }
   }
 }
@@ -121,9 +153,9 @@ unsigned grid_for(uint64_t n_vec) {
 }  // namespace
 
 cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, int64_t n_rows, int hidden,
-                            const BlockTable& bt, dp_dtype dt, cudaStream_t s) {
+                            const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s) {
   if (nseg < 1 || nseg > 2 || n_rows <= 0) return cudaErrorInvalidValue;
-  const int eb = dt == DP_BF16 ? 2 : 4;
+  const int eb = x_dt == DP_F32 ? 4 : 2;
   const uint64_t vpr = static_cast<uint64_t>(hidden) * eb / 16;
   const uint64_t vps = vpr * static_cast<uint64_t>(n_rows);
   if (vps >= (1ull << 31)) return cudaErrorInvalidValue;
@@ -134,10 +166,17 @@ cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, 
     segs.dst[i] = static_cast<uint4*>(dst[j]);
   }
   dim3 grid(grid_for(vps), nseg);
-  if (dt == DP_BF16)
-    modulate_kernel<true><<<grid, kThreads, 0, s>>>(segs, static_cast<uint32_t>(vpr), static_cast<uint32_t>(vps), hidden, bt);
+  const uint32_t a = static_cast<uint32_t>(vpr), b = static_cast<uint32_t>(vps);
+  if (x_dt == DP_BF16 && y_dt == DP_BF16)
+    modulate_kernel<kBF16, kBF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+  else if (x_dt == DP_BF16 && y_dt == DP_F16)
+    modulate_kernel<kBF16, kF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+  else if (x_dt == DP_F16 && y_dt == DP_F16)
+    modulate_kernel<kF16, kF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+  else if (x_dt == DP_F32 && y_dt == DP_F32)
+    modulate_kernel<kF32, kF32><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
   else
-    modulate_kernel<false><<<grid, kThreads, 0, s>>>(segs, static_cast<uint32_t>(vpr), static_cast<uint32_t>(vps), hidden, bt);
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

@@ -77,9 +77,10 @@ def modulate(x, row_offset: Sequence[int], mod) -> np.ndarray:
 
 
 def modulate_rounded(x, row_offset: Sequence[int], mod, dtype: str) -> np.ndarray:
-    """The modulated features as stored in ``dtype``: 1 + scale is formed in float32, the
-    product and sum are exact in float64 (8-bit x 24-bit significands), then the value is
-    rounded once to float32 and once more to the storage type (round to nearest even).
+    """The modulated features as stored in ``dtype`` ("f32", "bf16" or "f16"): 1 + scale is
+    formed in float32, the product and sum are exact in float64 (at most 11-bit x 24-bit
+    significands), then the value is rounded once to float32 and once more to the storage
+    type (round to nearest even; f16 saturates at +-65504 instead of overflowing).
     Returns the stored values as float64."""
     import torch
     x = as_f64(x)
@@ -92,6 +93,8 @@ def modulate_rounded(x, row_offset: Sequence[int], mod, dtype: str) -> np.ndarra
         return y32.to(torch.float64).numpy()
     if dtype == "bf16":
         return y32.to(torch.bfloat16).to(torch.float64).numpy()
+    if dtype == "f16":
+        return y32.clamp(-65504.0, 65504.0).to(torch.float16).to(torch.float64).numpy()
     raise ValueError(dtype)
 
 

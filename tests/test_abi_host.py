@@ -99,11 +99,11 @@ def test_blocks_from_table_checks(m):
 
 
 def _attn(m, q=FAKE, k=FAKE + 1024, v=FAKE + 2048, n=256, ck=FAKE + 4096, cv=FAKE + 8192, lc=128,
-          out=FAKE + 16384, H=2, hd=64, blk=None, dt=1):
+          out=FAKE + 16384, H=2, hd=64, blk=None, dt=1, ft=2):
     blk = blk if blk is not None else _blocks(m, [128, 128], H * hd)
     return m._lib.dp_window_attention(ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v), n,
                                       ctypes.c_void_p(ck), ctypes.c_void_p(cv), lc, None, ctypes.c_void_p(out),
-                                      H, hd, 0.0, ctypes.byref(blk), 3, dt, None)
+                                      H, hd, 0.0, ctypes.byref(blk), 3, dt, ft, None)
 
 
 def test_attention_argument_errors(m):
@@ -111,7 +111,9 @@ def test_attention_argument_errors(m):
     assert _attn(m, q=FAKE + 8) == m.ERR_INVALID_ARG                # misaligned
     assert _attn(m, n=0, blk=_blocks(m, [0], 128)) == m.ERR_INVALID_ARG
     assert _attn(m, H=1, hd=96, blk=_blocks(m, [128, 128], 96)) == m.ERR_UNSUPPORTED
-    assert _attn(m, H=1, hd=96, dt=0, blk=_blocks(m, [128, 128], 96)) == m.ERR_UNSUPPORTED
+    assert _attn(m, H=1, hd=96, dt=0, ft=0, blk=_blocks(m, [128, 128], 96)) == m.ERR_UNSUPPORTED
+    assert _attn(m, dt=0, ft=2) == m.ERR_UNSUPPORTED              # f32 window with f16 features
+    assert _attn(m, dt=2, ft=2) == m.ERR_UNSUPPORTED              # f16 window
     assert _attn(m, blk=_blocks(m, [128, 127], 128)) == m.ERR_INVALID_ARG   # offsets != n_win
     assert _attn(m, out=FAKE) == m.ERR_INVALID_ARG                  # out aliases q
     assert _attn(m, lc=-1) == m.ERR_INVALID_ARG
@@ -123,7 +125,16 @@ def test_attention_argument_errors(m):
     assert _attn(m, dt=7) == m.ERR_INVALID_ARG
 
 
-def _cache(m, capacity=128, hidden=128, n_slots=1, length=0, dt=1):
+def test_modulate_dtype_pairs(m):
+    blk = _blocks(m, [8], 64)
+    mod = lambda xd, yd: m._lib.dp_adaln_modulate(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 4096), 8,
+                                                  ctypes.byref(blk), xd, yd, None)
+    assert mod(0, 2) == m.ERR_UNSUPPORTED        # f32 -> f16
+    assert mod(2, 1) == m.ERR_UNSUPPORTED        # f16 -> bf16
+    assert mod(1, 5) == m.ERR_INVALID_ARG
+
+
+def _cache(m, capacity=128, hidden=128, n_slots=1, length=0, dt=2):
     c = m.DpKvcache()
     c.k, c.v = FAKE + (1 << 20), FAKE + (2 << 20)
     c.capacity, c.hidden, c.n_slots, c.dtype = capacity, hidden, n_slots, dt
@@ -187,6 +198,10 @@ def test_queue_blocks_host_lookup(m):
 def test_window_step_checks_before_launch(m):
     blk = _blocks(m, [128, 128], 128)
     c = _cache(m, capacity=100)
+    assert m._lib.dp_window_step(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), 256,
+                                 ctypes.byref(blk), ctypes.byref(_cache(m, dt=1)), ctypes.c_void_p(FAKE + (64 << 20)),
+                                 None, ctypes.c_void_p(FAKE + (32 << 20)), 2, 64, 0, None, None, 0, 1,
+                                 None) == m.ERR_INVALID_ARG     # bf16 window needs an f16 feature cache
     args = lambda flags, queue=None, noise=None, rows=0: m._lib.dp_window_step(
         ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), 256, ctypes.byref(blk), ctypes.byref(c),
         ctypes.c_void_p(FAKE + (64 << 20)), None, ctypes.c_void_p(FAKE + (32 << 20)), 2, 64, flags,

@@ -27,10 +27,10 @@ def test_long_run_matches_oracle(dp):
     tau = O.timestep_schedule(T)
     run = O.LongRun(noise_cpu, table_cpu, H, hd, W, T)
     total = len(run.schedule)
-    cache = dp.KVCache(rc.slot_rows, D, torch.bfloat16)
+    cache = dp.KVCache(rc.slot_rows, D, torch.float16)
     queue = dp.Queue(W, rc.slot_rows, D)
     n_max = W * rc.slot_rows
-    kv = torch.empty(2, n_max, D, dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty(2 * n_max * D, dtype=torch.float16, device="cuda")  # k' then v' at n_win * D
     out = torch.empty(n_max, D, dtype=torch.bfloat16, device="cuda")
     m_last = O.lookup(table_cpu, [tau[T - 1]])
     live = [0]
@@ -39,6 +39,7 @@ def test_long_run_matches_oracle(dp):
 
     def on_step(step, n, popped, pushed):
         sched = run.schedule[step]
+        kp, vp = kv[:n * D].view(n, D), kv[n * D:2 * n * D].view(n, D)
         assert live == sched["live"], (step, live, sched["live"])
         assert n == sum(noise_cpu[b].shape[0] for b in live)
         if step in CHECK_STEPS:
@@ -54,10 +55,10 @@ def test_long_run_matches_oracle(dp):
             torch.cuda.synchronize()
             # the cache is the exited block's k'/v' from this (its last) evaluation
             assert cache.length == n_exit
-            assert bytes_equal(cache.k[0, :n_exit], kv[0, :n_exit])
-            assert bytes_equal(cache.v[0, :n_exit], kv[1, :n_exit])
+            assert bytes_equal(cache.k[0, :n_exit], kp[:n_exit])
+            assert bytes_equal(cache.v[0, :n_exit], vp[:n_exit])
             if len(advances) % 16 == 0 or b == len(noise_cpu) - 1:
-                want = O.modulate_rounded(noise_cpu[b], [0, n_exit], m_last, "bf16")
+                want = O.modulate_rounded(noise_cpu[b], [0, n_exit], m_last, "f16")
                 assert np.array_equal(cache.k[0, :n_exit].cpu().double().numpy(), want)
             advances.append(b)
         else:

@@ -6,7 +6,9 @@ import torch
 
 import oracle as O
 from tests.gpu_util import assert_close, bytes_equal, errors, sample_rows
-from workloads import make_step_inputs, step_config, to_dtype
+from workloads import as_features, make_step_inputs, step_config, to_dtype
+
+TDT = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -24,16 +26,17 @@ def _randn(shape, seed, dtype, std=1.0):
 
 # --------------------------------------------------------------------------- A1 modulation
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtypes", [("bf16", "f16"), ("bf16", "bf16"), ("f32", "f32")])
 @pytest.mark.parametrize("rows", [[300, 450, 250], [1], [0, 7, 129, 0]])
-def test_modulate_matches_oracle_bitwise(dp, dtype, rows):
+def test_modulate_matches_oracle_bitwise(dp, dtypes, rows):
+    x_dt, dtype = dtypes
     D = 1536
     n = sum(rows)
-    x = _randn((n, D), 1, dtype)
+    x = _randn((n, D), 1, x_dt)
     table = _table(D)
     ts = [int(t) for t in np.linspace(0, 999, len(rows)).round()]
     xd, td = x.cuda(), table.cuda()
-    y = torch.empty_like(xd)
+    y = torch.empty(n, D, dtype=TDT[dtype], device="cuda")
     blk = dp.blocks_from_table(td, ts, rows)
     dp.adaln_modulate(xd, y, blk)
     ro = blk.offsets
@@ -47,35 +50,38 @@ def test_modulate_matches_oracle_bitwise(dp, dtype, rows):
     exact = O.modulate(x, ro, mod)
     beta = O.row_blocks(ro, n)
     xf = O.as_f64(x)
-    u = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -24
+    u = {"bf16": 2.0 ** -8, "f16": 2.0 ** -11, "f32": 2.0 ** -24}[dtype]
     bound = u * np.abs(exact) + 2.0 ** -22 * (np.abs(xf * (1.0 + mod[beta, 1])) + np.abs(mod[beta, 0]))
     assert np.all(np.abs(got - exact) <= bound)
-    # in place gives the same bytes
-    dp.adaln_modulate(xd, xd, blk)
-    assert bytes_equal(xd, y)
+    if x_dt == dtype:                       # in place gives the same bytes
+        dp.adaln_modulate(xd, xd, blk)
+        assert bytes_equal(xd, y)
 
 
 # --------------------------------------------------------------------------- A2 attention
 
 ATTN_CASES = [
-    # (H, hd, block rows, cache_len, cache capacity, residual, flags)
-    (2, 64, [500, 300, 200], 300, 333, False, 3),
-    (2, 128, [400, 377], 0, 16, True, 3),
-    (3, 64, [129], 1, 8, False, 3),
-    (1, 64, [1], 0, 1, False, 3),
-    (2, 128, [256, 256], 128, 128, True, 0),
-    (4, 64, [100, 0, 156, 1], 200, 256, True, 1),
-    (2, 64, [5000], 2500, 2500, False, 2),
+    # (H, hd, block rows, cache_len, cache capacity, residual, flags, feature dtype)
+    (2, 64, [500, 300, 200], 300, 333, False, 3, "f16"),
+    (2, 128, [400, 377], 0, 16, True, 3, "f16"),
+    (3, 64, [129], 1, 8, False, 3, "f16"),
+    (1, 64, [1], 0, 1, False, 3, "f16"),
+    (2, 128, [256, 256], 128, 128, True, 0, "f16"),
+    (4, 64, [100, 0, 156, 1], 200, 256, True, 1, "f16"),
+    (2, 64, [5000], 2500, 2500, False, 2, "f16"),
+    (2, 64, [700, 300], 300, 300, False, 3, "bf16"),
+    (2, 128, [257, 255], 100, 100, True, 3, "bf16"),
 ]
 
 
-@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"H{c[0]}_hd{c[1]}_n{sum(c[2])}_c{c[3]}")
+@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"H{c[0]}_hd{c[1]}_n{sum(c[2])}_c{c[3]}_{c[7]}")
 def test_attention_bf16_matches_oracle(dp, case):
-    H, hd, rows, Lc, cap, with_res, flags = case
+    H, hd, rows, Lc, cap, with_res, flags, ft = case
     D = H * hd
     n = sum(rows)
-    q, k, v = (_randn((n, D), s, "bf16") for s in (11, 12, 13))
-    ck, cv = (_randn((cap, D), s, "bf16") for s in (14, 15))
+    q = _randn((n, D), 11, "bf16")
+    k, v = (_randn((n, D), s, "bf16").to(TDT[ft]) for s in (12, 13))
+    ck, cv = (_randn((cap, D), s, "bf16").to(TDT[ft]) for s in (14, 15))
     res = _randn((n, D), 16, "bf16") if with_res else None
     table = _table(D)
     ts = [int(t) for t in np.linspace(0, 999, len(rows)).round()]
@@ -92,7 +98,8 @@ def test_attention_bf16_matches_oracle(dp, case):
 def test_attention_bf16_deterministic(dp):
     H, hd, n, Lc = 4, 64, 1000, 300
     D = H * hd
-    q, k, v, ck, cv = (_randn((n, D), s, "bf16").cuda() for s in range(5))
+    q = _randn((n, D), 0, "bf16").cuda()
+    k, v, ck, cv = (_randn((n, D), s, "bf16").to(torch.float16).cuda() for s in range(1, 5))
     blk = dp.blocks_from_table(_table(D).cuda(), [0, 500], [600, 400])
     a = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
     b = torch.empty_like(a)
@@ -208,23 +215,24 @@ def test_window_step_full_size_sampled(dp, name):
     x = make_step_inputs(cfg)
     H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
     blk = dp.blocks_from_table(x["table"].cuda(), x["timesteps"], cfg.block_rows)
-    cache = dp.KVCache(cfg.cache_capacity, D, torch.bfloat16, k=x["cache_k"].cuda().view(1, -1, D),
-                       v=x["cache_v"].cuda().view(1, -1, D), length=cfg.cache_len)
+    ck, cv = as_features(x["cache_k"], cfg.dtype), as_features(x["cache_v"], cfg.dtype)
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.float16, k=ck.cuda().view(1, -1, D),
+                       v=cv.cuda().view(1, -1, D), length=cfg.cache_len)
     qu = dp.Queue(cfg.n_blocks, cfg.block_rows[0], D)
     for _ in range(cfg.n_blocks):
         dp.queue_push(qu, x["noise"].cuda())
-    kv = torch.empty(2, n, D, dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty(2, n, D, dtype=torch.float16, device="cuda")
     out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
     dp.window_step(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), blk, cache, kv, out, H, hd, pop=True, queue=qu,
                    push_noise=x["noise"].cuda())
     dp.device_status()
     rows = sample_rows(cfg.row_offset, n_extra=64)
     mod = O.lookup(x["table"], x["timesteps"])
-    want, _, _ = O.window_step(x["q"], x["k"], x["v"], x["cache_k"], x["cache_v"], cfg.cache_len, cfg.row_offset,
+    want, _, _ = O.window_step(x["q"], x["k"], x["v"], ck, cv, cfg.cache_len, cfg.row_offset,
                                mod, H, hd, rows=rows)
     got = out[rows].cpu().double().numpy()
     assert_close(got, want, "bf16", name)
     n0 = cfg.block_rows[0]
     assert bytes_equal(cache.k[0, :n0], kv[0, :n0]) and bytes_equal(cache.v[0, :n0], kv[1, :n0])
-    kr = O.modulate_rounded(x["k"][:n0], [0, n0], mod[:1], "bf16")
+    kr = O.modulate_rounded(x["k"][:n0], [0, n0], mod[:1], "f16")
     assert np.array_equal(cache.k[0, :n0].cpu().double().numpy(), kr)

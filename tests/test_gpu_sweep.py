@@ -8,7 +8,7 @@ import torch
 
 import oracle as O
 from tests.gpu_util import assert_close, bytes_equal, sample_rows
-from workloads import make_step_inputs, step_config
+from workloads import as_features, make_step_inputs, step_config
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -18,14 +18,15 @@ def _run(dp, cfg):
     x = make_step_inputs(cfg)
     H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
     blk = dp.blocks_from_table(x["table"].cuda(), x["timesteps"], cfg.block_rows)
-    cache = dp.KVCache(cfg.cache_capacity, D, torch.bfloat16, k=x["cache_k"].cuda().view(1, -1, D),
+    x["cache_k"], x["cache_v"] = as_features(x["cache_k"], cfg.dtype), as_features(x["cache_v"], cfg.dtype)
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.float16, k=x["cache_k"].cuda().view(1, -1, D),
                        v=x["cache_v"].cuda().view(1, -1, D), length=cfg.cache_len)
-    kv = torch.empty(2, n, D, dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty(2, n, D, dtype=torch.float16, device="cuda")
     out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
     dp.window_step(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), blk, cache, kv, out, H, hd, pop=True)
     dp.device_status()
     n0 = cfg.block_rows[0]
-    assert cache.length == n0 and bytes_equal(cache.k[0, :n0], kv[0, :n0])
+    assert cache.length == n0 and bytes_equal(cache.k[0, :n0], kv[0, :n0]) and bytes_equal(cache.v[0, :n0], kv[1, :n0])
     return x, out
 
 

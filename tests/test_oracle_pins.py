@@ -68,6 +68,16 @@ def test_modulate_rounded_hand_cases():
     assert y.tolist() == [[1.75, 1.0, 1.0 + 2.0 ** -7, -1.5]]
 
 
+def test_modulate_rounded_f16_hand_cases():
+    # f16 has 10 fraction bits: 1 + 2^-11 is a tie and rounds to even (1.0); 1 + 3 * 2^-12
+    # rounds up to 1 + 2^-10; 60000 * 2 saturates at 65504 instead of overflowing
+    x = np.array([[1.0, 1.0, 60000.0, -60000.0]])
+    mod = np.zeros((1, 3, 4))
+    mod[0, 1] = [2.0 ** -11, 3 * 2.0 ** -12, 1.0, 1.0]
+    y = O.modulate_rounded(x, [0, 1], mod, "f16")
+    assert y.tolist() == [[1.0, 1.0 + 2.0 ** -10, 65504.0, -65504.0]]
+
+
 def test_modulate_rounded_within_one_bf16_rounding():
     rng = _rng(3)
     x = torch.randn(64, 32, dtype=torch.float32).to(torch.bfloat16)

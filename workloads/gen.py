@@ -23,6 +23,12 @@ def to_dtype(x: torch.Tensor, dtype: str) -> torch.Tensor:
     raise ValueError(dtype)
 
 
+def as_features(x: torch.Tensor, dtype: str) -> torch.Tensor:
+    """Cached K/V enter the window step as stored features: f16 on the bf16 path (every bf16
+    value in f16's normal range converts exactly), fp32 on the fp32 path."""
+    return x.to(torch.float16).contiguous() if dtype == "bf16" else x.to(torch.float32).contiguous()
+
+
 def _randn(g: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
     x = torch.randn(*shape, generator=g, dtype=torch.float32)
     if std != 1.0:
