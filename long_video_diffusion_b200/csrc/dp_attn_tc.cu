@@ -65,17 +65,24 @@ struct Layout {
   static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 B
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
+  // Tensor memory: S_g (BN fp32 columns each), P_g (BN/2 columns of 16-bit pairs), O_g (HD
+  // columns).  When all of it fits, P has its own columns and the next S product can run
+  // while the softmax still works on the current tile; otherwise P is written over S_g.
+  static constexpr bool SEP_P = 2 * BN + 2 * (BN / 2) + 2 * HD <= kTmemCols;
+  static constexpr int COL_P = SEP_P ? 2 * BN : 0;
+  static constexpr int P_STRIDE = SEP_P ? BN / 2 : BN;
+  static constexpr int COL_O = SEP_P ? 3 * BN : 2 * BN;
+  static_assert(COL_O + NQ * HD <= kTmemCols, "tensor memory budget");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  // k_full[S], v_full[S], kv_empty[S], q_full[2], s_full[2], p_full[2], o_done[2], fin
-  static constexpr int N_BAR = 3 * STAGES + 4 * NQ + 1;
+  // k_full[S], v_full[S], kv_empty[S], q_full[2], s_full[2], s_free[2], p_full[2], o_done[2], fin
+  static constexpr int N_BAR = 3 * STAGES + 5 * NQ + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;             // room to align the base to 1 KB
   static_assert(ALLOC <= 227 * 1024, "shared memory budget");
-  static_assert(256 + NQ * HD <= kTmemCols, "tensor memory budget");
 };
 
 struct Params {
@@ -110,8 +117,8 @@ __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_ca
 template <int HD, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     window_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
-                     const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
-                     const Params p) {
+                          const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
+                          const Params p) {
   using L = Layout<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,9 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto kv_empty = [&](int s) { return bar0 + 8u * (2 * L::STAGES + s); };
   auto q_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + g); };
   auto s_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + NQ + g); };
-  auto p_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 2 * NQ + g); };
-  auto o_done = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 3 * NQ + g); };
-  const uint32_t fin = bar0 + 8u * (3 * L::STAGES + 4 * NQ);
+  auto s_free = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 2 * NQ + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 3 * NQ + g); };
+  auto o_done = [&](int g) { return bar0 + 8u * (3 * L::STAGES + 4 * NQ + g); };
+  const uint32_t fin = bar0 + 8u * (3 * L::STAGES + 5 * NQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -143,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < NQ; ++g) {
       mbar_init(q_full(g), 128);
       mbar_init(s_full(g), 1);
+      mbar_init(s_free(g), 128);
       mbar_init(p_full(g), 128);
       mbar_init(o_done(g), 1);
     }
@@ -198,6 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Polls both query tiles' barriers and issues whichever product is ready, so neither
+    // softmax warpgroup waits for the other:
+    //   S_g(t) = Q_g K_t^T   needs K_t, and S_g(t-1) consumed (read by the softmax when P
+    //                        has its own columns; else PV_g(t-1) issued, since MMAs from
+    //                        this thread execute in issue order and P_g(t-1) lives in S_g)
+    //   O_g += P_g(t) V_t    needs P_g(t) and V_t
+    // The K/V stage of tile t is released once both query tiles' PV(t) are issued.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f32acc(Operand<F16>::kFmt, BM, BN, false);
       constexpr uint32_t idPV = idesc_f32acc(Operand<F16>::kFmt, BM, HD, true);
@@ -207,53 +223,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + g * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+          mma_ss(tmem + g * BN, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
         }
       };
       auto issue_pv = [&](int g, int st, bool acc) {
         const uint32_t va = sb + L::OFF_V + st * L::KV_BYTES;
+        const uint32_t pa = tmem + L::COL_P + g * L::P_STRIDE;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tmem + 256 + g * HD, tmem + g * 128 + kk * 8, sdesc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), idPV,
+          mma_ts(tmem + L::COL_O + g * HD, pa + kk * 8, sdesc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), idPV,
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(q_full(0), 0, abort, p.status, DEV_ERR_TIMEOUT_Q) &&
-                mbar_wait(q_full(1), 0, abort, p.status, DEV_ERR_TIMEOUT_Q) &&
-                mbar_wait(k_full(0), 0, abort, p.status, DEV_ERR_TIMEOUT_KV);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(s_full(0));
-        issue_s(1, 0);
-        mma_commit(s_full(1));
-      }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % L::STAGES;
-        if (!mbar_wait(v_full(st), (j / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV)) break;
-        for (int g = 0; g < NQ && ok; ++g) {
-          if (!mbar_wait(p_full(g), j & 1, abort, p.status, DEV_ERR_TIMEOUT_P)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(g, st, j > 0);
-          mma_commit(o_done(g));
-          if (g == NQ - 1) mma_commit(kv_empty(st));
-          if (j + 1 < n_tiles) {
-            const int st1 = (j + 1) % L::STAGES;
-            if (g == 0) {
-              if (!mbar_wait(k_full(st1), ((j + 1) / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV)) {
-                ok = false;
-                break;
-              }
+                mbar_wait(q_full(1), 0, abort, p.status, DEV_ERR_TIMEOUT_Q);
+      if (ok) tc_fence_after();
+      int ns[NQ] = {0, 0};  // next S tile per query tile
+      int np[NQ] = {0, 0};  // next PV tile per query tile
+      uint64_t t_last = globaltimer();
+      while (ok && (np[0] < n_tiles || np[1] < n_tiles)) {
+        bool progress = false;
+#pragma unroll
+        for (int g = 0; g < NQ; ++g) {
+          const int ts = ns[g];
+          if (ts < n_tiles) {
+            bool ready = ts == 0 || (L::SEP_P ? mbar_try_wait(s_free(g), (ts - 1) & 1) : np[g] >= ts);
+            ready = ready && mbar_try_wait(k_full(ts % L::STAGES), (ts / L::STAGES) & 1);
+            if (ready) {
               tc_fence_after();
+              issue_s(g, ts % L::STAGES);
+              mma_commit(s_full(g));
+              ns[g] = ts + 1;
+              progress = true;
             }
-            // S(g) of the next tile overwrites P(g) of this tile: the MMAs issued by this
-            // thread execute in issue order, so the PV product above has read P first.
-            issue_s(g, st1);
-            mma_commit(s_full(g));
           }
+          const int tp = np[g];
+          if (tp < ns[g] && mbar_try_wait(p_full(g), tp & 1) &&
+              mbar_try_wait(v_full(tp % L::STAGES), (tp / L::STAGES) & 1)) {
+            tc_fence_after();
+            issue_pv(g, tp % L::STAGES, tp > 0);
+            mma_commit(o_done(g));
+            np[g] = tp + 1;
+            if (np[1 - g] > tp) mma_commit(kv_empty(tp % L::STAGES));
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = globaltimer();
+        } else if (*abort) {
+          break;
+        } else if (globaltimer() - t_last > kWaitLimitNs) {
+          atomicOr(p.status, DEV_ERR_TIMEOUT_P);
+          *abort = 1;
+          break;
         }
       }
       mma_commit(fin);
@@ -308,8 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     const uint32_t trow = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
-    const uint32_t s_col = g * 128;
-    const uint32_t o_col = 256 + g * HD;
+    const uint32_t s_col = g * BN;
+    const uint32_t p_col = L::COL_P + g * L::P_STRIDE;
+    const uint32_t o_col = L::COL_O + g * HD;
+    const uint64_t sl2 = f32x2(p.scale_log2, p.scale_log2);
     float m_ref = -INFINITY;
     float l_sum = 0.0f;
     bool ok = true;
@@ -323,30 +347,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) tmem_ld32(trow + s_col + i * 32, sr[i]);
       tmem_wait_ld();
+      if constexpr (L::SEP_P) {
+        // S is in registers: the tensor core may overwrite it with the next tile's S
+        tc_fence_before();
+        mbar_arrive(s_free(g));
+      }
       const int64_t key0 = (j < p.n_ct) ? static_cast<int64_t>(j) * BN : static_cast<int64_t>(j - p.n_ct) * BN;
-      const int64_t seg_len = (j < p.n_ct) ? p.cache_len : p.n_win;
-      const int64_t rem = seg_len - key0;
-      const int valid = rem < BN ? static_cast<int>(rem) : BN;
-      float mx = -INFINITY;
+      const int64_t rem = ((j < p.n_ct) ? p.cache_len : p.n_win) - key0;
+      if (rem < BN) {  // last tile of a segment: keys beyond it get -inf (TMA filled them with 0)
+        const int valid = static_cast<int>(rem);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (i * 32 + c >= valid) sr[i][c] = 0xff800000u;
+      }
+      // row max: four independent chains of 3-input max
+      float mc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        float m = fmaxf(__uint_as_float(sr[i][0]), __uint_as_float(sr[i][31]));
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (i * 32 + c >= valid) sr[i][c] = 0xff800000u;  // -inf: key beyond the segment
-          mx = fmaxf(mx, __uint_as_float(sr[i][c]));
-        }
+        for (int c = 1; c < 31; c += 2) m = fmax3(m, __uint_as_float(sr[i][c]), __uint_as_float(sr[i][c + 1]));
+        mc[i] = m;
       }
+      const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]);
       const float m_new = fmaxf(m_ref, mx * p.scale_log2);
       if (j == 0) {
         m_ref = m_new;
       } else {
         const bool need = m_new > m_ref + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          // the previous PV product must be complete before O is read and rescaled
+        const bool any_need = __any_sync(0xffffffffu, need);
+        if (L::SEP_P || any_need) {
+          // PV(j-1) must be complete before O is rescaled or P(j-1) is overwritten
           ok = mbar_wait(o_done(g), (j - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
+        }
+        if (any_need) {
           const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
 #pragma unroll
           for (int c0 = 0; c0 < HD; c0 += 32) {
@@ -364,18 +403,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      const float nm = -m_ref;
+      // P = exp2(s * scale * log2(e) - m_ref): packed FMA, MUFU exp2, packed adds
+      const uint64_t nm2 = f32x2(-m_ref, -m_ref);
+      uint64_t acc0 = f32x2(0.0f, 0.0f), acc1 = acc0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float a = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c]), p.scale_log2, nm));
-          const float b = ex2_approx(fmaf(__uint_as_float(sr[i][2 * c + 1]), p.scale_log2, nm));
-          l_sum += a + b;
-          pk[c] = Operand<F16>::pack(a, b);
+          const uint64_t x = ffma2(f32x2(__uint_as_float(sr[i][2 * c]), __uint_as_float(sr[i][2 * c + 1])), sl2, nm2);
+          float x0, x1;
+          f32x2_split(x, x0, x1);
+          const float a = ex2_approx(x0);
+          const float b = ex2_approx(x1);
+          const uint64_t ab = f32x2(a, b);
+          if (c & 1)
+            acc1 = fadd2(acc1, ab);
+          else
+            acc0 = fadd2(acc0, ab);
+          pk[c] = Operand<F16>::pack_p(a, b);
         }
-        tmem_st16(trow + s_col + i * 16, pk);
+        tmem_st16(trow + p_col + i * 16, pk);
+      }
+      {
+        const uint64_t acc = fadd2(acc0, acc1);
+        float a0, a1;
+        f32x2_split(acc, a0, a1);
+        l_sum += a0 + a1;
       }
       tmem_wait_st();
       tc_fence_before();

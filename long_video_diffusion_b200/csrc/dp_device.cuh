@@ -246,16 +246,60 @@ __device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
   return r;
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // 16-bit tensor-core operand type: F16 = true selects f16 (11-bit significand), else bf16.
 template <bool F16>
 struct Operand {
   static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor A/B format
+  // features (may be large): f16 saturates instead of overflowing
   __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
     if constexpr (F16)
       return pack_f16x2_sat(lo, hi);
     else
       return pack_bf16x2(lo, hi);
   }
+  // softmax weights, in (0, 256]: plain round to nearest even
+  __device__ __forceinline__ static uint32_t pack_p(float lo, float hi) {
+    if constexpr (F16)
+      return pack_f16x2(lo, hi);
+    else
+      return pack_bf16x2(lo, hi);
+  }
 };
+
+// ------------------------------------------------------------------ packed fp32 pairs
+
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 }  // namespace dp

@@ -3,9 +3,7 @@
 // Modulation (each block conditioned on its own timestep: "Minute-Long Videos with Dual
 // Parallelisms", abstract, blocks at progressively decreasing noise levels; pith.science
 // review, Section 3.1): y = x * (1 + scale_b) + shift_b per channel, one fp32 FMA per
-// element, rounded once to the output type (f16 saturates at +-65504).  Each thread moves 16-byte vectors (8 bf16
-// or 4 fp32) with four independent vectors in flight; the grid is a multiple of the SM
-// count and strides over all rows of every segment.
+// element, rounded once to the output type (f16 saturates at +-65504).
 //
 // Copy (the queue advance: the exiting block's K'/V' rows become the cache, a fresh noise
 // block enters the latent ring; review, key machinery and Section 3.2): up to four
@@ -23,11 +21,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
-
-struct ModSegs {
-  const uint4* src[2];
-  uint4* dst[2];
-};
 
 // Element formats of a 16-byte vector: 8 bf16, 8 f16 or 4 fp32.
 enum Fmt { kBF16 = 0, kF16 = 1, kF32 = 2 };
@@ -70,46 +63,52 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   }
 }
 
-// y = x * (1 + scale) + shift on one 16-byte vector; 1 + scale formed in fp32, one FMA.
-template <int FI, int FO>
-__device__ __forceinline__ uint4 mod_vec(uint4 x, const float* sh, const float* sc) {
-  constexpr int VE = FI == kF32 ? 4 : 8;
-  float f[8], shv[8], scv[8];
-  unpack8<FI>(x, f);
-#pragma unroll
-  for (int v = 0; v < VE / 4; ++v) {
-    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sh) + v);
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(sc) + v);
-    shv[4 * v] = s4.x, shv[4 * v + 1] = s4.y, shv[4 * v + 2] = s4.z, shv[4 * v + 3] = s4.w;
-    scv[4 * v] = c4.x, scv[4 * v + 1] = c4.y, scv[4 * v + 2] = c4.z, scv[4 * v + 3] = c4.w;
-  }
-#pragma unroll
-  for (int e = 0; e < VE; ++e) f[e] = fmaf(f[e], 1.0f + scv[e], shv[e]);
-  return pack8<FO>(f);
-}
+// One CTA thread per 16-byte column vector of a row (blockDim = vectors per row, up to
+// 1024; wider rows loop); the CTA walks rows kRowsInFlight at a time, grid-striding over the
+// rows of its segment (grid.y).  A thread keeps its columns' shift and 1 + scale in
+// registers and reloads them only when the row's block changes, so HBM traffic is the 16
+// bytes read and written per vector and nothing else.
+constexpr int kRowsInFlight = 4;
 
 template <int FI, int FO>
-__global__ void __launch_bounds__(kThreads) modulate_kernel(ModSegs segs, uint32_t vec_per_row, uint32_t vec_per_seg,
-                                                            int hidden, BlockTable bt) {
+__global__ void __launch_bounds__(1024) modulate_kernel(const uint4* __restrict__ src0, uint4* __restrict__ dst0,
+                                                        const uint4* __restrict__ src1, uint4* __restrict__ dst1,
+                                                        uint32_t n_rows, uint32_t vec_per_row, int hidden,
+                                                        BlockTable bt) {
   constexpr int VE = FI == kF32 ? 4 : 8;  // elements per 16-byte vector
-  const uint4* src = segs.src[blockIdx.y];
-  uint4* dst = segs.dst[blockIdx.y];
-  const uint32_t stride = gridDim.x * kThreads;
-  for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < vec_per_seg; base += stride * kUnroll) {
-    uint4 x[kUnroll];
-    uint32_t idx[kUnroll];
+  const uint4* src = blockIdx.y ? src1 : src0;
+  uint4* dst = blockIdx.y ? dst1 : dst0;
+  for (uint32_t cv = threadIdx.x; cv < vec_per_row; cv += blockDim.x) {
+    const uint32_t col = cv * VE;
+    int cur = -1;
+    float sh[VE], a[VE];
+    for (uint32_t r0 = blockIdx.x * kRowsInFlight; r0 < n_rows; r0 += gridDim.x * kRowsInFlight) {
+      uint4 x[kRowsInFlight];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      idx[u] = base + u * stride;
-      if (idx[u] < vec_per_seg) x[u] = __ldcs(src + idx[u]);
-    }
+      for (int u = 0; u < kRowsInFlight; ++u)
+        if (r0 + u < n_rows) x[u] = __ldcs(src + static_cast<size_t>(r0 + u) * vec_per_row + cv);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (idx[u] >= vec_per_seg) break;
-      const uint32_t row = idx[u] / vec_per_row;
-      const uint32_t col = (idx[u] - row * vec_per_row) * VE;
-      const float* m = block_mod(bt, block_of_row(bt, row));
-      dst[idx[u]] = mod_vec<FI, FO>(x[u], m + col, m + hidden + col);
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const uint32_t row = r0 + u;
+        if (row >= n_rows) break;
+        const int b = block_of_row(bt, row);
+        if (b != cur) {
+          const float* m = block_mod(bt, b);
+#pragma unroll
+          for (int v = 0; v < VE / 4; ++v) {
+            const float4 s4 = __ldg(reinterpret_cast<const float4*>(m + col) + v);
+            const float4 c4 = __ldg(reinterpret_cast<const float4*>(m + hidden + col) + v);
+            sh[4 * v] = s4.x, sh[4 * v + 1] = s4.y, sh[4 * v + 2] = s4.z, sh[4 * v + 3] = s4.w;
+            a[4 * v] = 1.0f + c4.x, a[4 * v + 1] = 1.0f + c4.y, a[4 * v + 2] = 1.0f + c4.z, a[4 * v + 3] = 1.0f + c4.w;
+          }
+          cur = b;
+        }
+        float f[8];
+        unpack8<FI>(x[u], f);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) f[e] = fmaf(f[e], a[e], sh[e]);
+        dst[static_cast<size_t>(row) * vec_per_row + cv] = pack8<FO>(f);
+      }
     }
   }
 }
@@ -121,9 +120,18 @@ struct CopySegs {
 };
 
 __global__ void __launch_bounds__(kThreads) copy_kernel(CopySegs segs) {
-  const uint4* src = segs.src[blockIdx.y];
-  uint4* dst = segs.dst[blockIdx.y];
-  const uint32_t n = segs.n_vec[blockIdx.y];
+  // segment selected with constant indices (no run-time indexing of the kernel argument)
+  const uint32_t y = blockIdx.y;
+  const uint4* src = segs.src[0];
+  uint4* dst = segs.dst[0];
+  uint32_t n = segs.n_vec[0];
+#pragma unroll
+  for (int i = 1; i < kMaxCopySegs; ++i)
+    if (y == static_cast<uint32_t>(i)) {
+      src = segs.src[i];
+      dst = segs.dst[i];
+      n = segs.n_vec[i];
+    }
   const uint32_t stride = gridDim.x * kThreads;
   for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < n; base += stride * kUnroll) {
     uint4 x[kUnroll];
@@ -154,27 +162,28 @@ unsigned grid_for(uint64_t n_vec) {
 
 cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, int64_t n_rows, int hidden,
                             const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s) {
-  if (nseg < 1 || nseg > 2 || n_rows <= 0) return cudaErrorInvalidValue;
+  if (nseg < 1 || nseg > 2 || n_rows <= 0 || n_rows >= (1ll << 31)) return cudaErrorInvalidValue;
   const int eb = x_dt == DP_F32 ? 4 : 2;
-  const uint64_t vpr = static_cast<uint64_t>(hidden) * eb / 16;
-  const uint64_t vps = vpr * static_cast<uint64_t>(n_rows);
-  if (vps >= (1ull << 31)) return cudaErrorInvalidValue;
-  ModSegs segs;
-  for (int i = 0; i < 2; ++i) {
-    const int j = i < nseg ? i : 0;
-    segs.src[i] = static_cast<const uint4*>(src[j]);
-    segs.dst[i] = static_cast<uint4*>(dst[j]);
-  }
-  dim3 grid(grid_for(vps), nseg);
-  const uint32_t a = static_cast<uint32_t>(vpr), b = static_cast<uint32_t>(vps);
+  const uint32_t vpr = static_cast<uint32_t>(static_cast<int64_t>(hidden) * eb / 16);
+  const unsigned threads = vpr >= 1024 ? 1024u : ((vpr + 31u) / 32u) * 32u;
+  // enough CTAs to fill every SM several times over, each with its own rows
+  const uint64_t row_groups = (static_cast<uint64_t>(n_rows) + kRowsInFlight - 1) / kRowsInFlight;
+  const uint64_t per_sm = 2048 / threads > 0 ? 2048 / threads : 1;
+  const uint64_t cap = static_cast<uint64_t>(sm_count()) * per_sm * 2;
+  dim3 grid(static_cast<unsigned>(row_groups < cap ? row_groups : cap), nseg);
+  const uint4* s0 = static_cast<const uint4*>(src[0]);
+  uint4* d0 = static_cast<uint4*>(dst[0]);
+  const uint4* s1 = static_cast<const uint4*>(src[nseg > 1 ? 1 : 0]);
+  uint4* d1 = static_cast<uint4*>(dst[nseg > 1 ? 1 : 0]);
+  const uint32_t nr = static_cast<uint32_t>(n_rows);
   if (x_dt == DP_BF16 && y_dt == DP_BF16)
-    modulate_kernel<kBF16, kBF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+    modulate_kernel<kBF16, kBF16><<<grid, threads, 0, s>>>(s0, d0, s1, d1, nr, vpr, hidden, bt);
   else if (x_dt == DP_BF16 && y_dt == DP_F16)
-    modulate_kernel<kBF16, kF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+    modulate_kernel<kBF16, kF16><<<grid, threads, 0, s>>>(s0, d0, s1, d1, nr, vpr, hidden, bt);
   else if (x_dt == DP_F16 && y_dt == DP_F16)
-    modulate_kernel<kF16, kF16><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+    modulate_kernel<kF16, kF16><<<grid, threads, 0, s>>>(s0, d0, s1, d1, nr, vpr, hidden, bt);
   else if (x_dt == DP_F32 && y_dt == DP_F32)
-    modulate_kernel<kF32, kF32><<<grid, kThreads, 0, s>>>(segs, a, b, hidden, bt);
+    modulate_kernel<kF32, kF32><<<grid, threads, 0, s>>>(s0, d0, s1, d1, nr, vpr, hidden, bt);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

@@ -44,14 +44,16 @@ def test_modulate_matches_oracle_bitwise(dp, dtypes, rows):
     want = O.modulate_rounded(x, ro, mod, dtype)
     got = y.cpu().double().numpy()
     assert np.array_equal(got, want), f"mismatches: {int((got != want).sum())}"
-    # against the float64 definition: one rounding to the storage type (unit roundoff u)
-    # plus the fp32 rounding of 1 + scale, which matters where x * (1 + scale) and shift
-    # nearly cancel
+    # against the float64 definition: one rounding to the storage type (unit roundoff u,
+    # plus half the smallest subnormal eta/2 for gradual underflow) and the fp32 rounding of
+    # 1 + scale, which matters where x * (1 + scale) and shift nearly cancel
     exact = O.modulate(x, ro, mod)
     beta = O.row_blocks(ro, n)
     xf = O.as_f64(x)
     u = {"bf16": 2.0 ** -8, "f16": 2.0 ** -11, "f32": 2.0 ** -24}[dtype]
-    bound = u * np.abs(exact) + 2.0 ** -22 * (np.abs(xf * (1.0 + mod[beta, 1])) + np.abs(mod[beta, 0]))
+    half_eta = {"bf16": 2.0 ** -134, "f16": 2.0 ** -25, "f32": 2.0 ** -150}[dtype]
+    bound = (u * np.abs(exact) + half_eta +
+             2.0 ** -22 * (np.abs(xf * (1.0 + mod[beta, 1])) + np.abs(mod[beta, 0])))
     assert np.all(np.abs(got - exact) <= bound)
     if x_dt == dtype:                       # in place gives the same bytes
         dp.adaln_modulate(xd, xd, blk)
