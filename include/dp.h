@@ -216,6 +216,33 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
                          uint32_t flags, dp_queue* queue, const void* push_noise,
                          int64_t push_rows, dp_dtype dt, void* stream);
 
+/* ---------------------------------------------------------------- step without allocation */
+
+/* Size in bytes of the fixed scratch array dp_window_step_noalloc uses on each device. */
+#define DP_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* dp_window_step without the kv_work argument, for callers that cannot allocate device
+ * memory: code embedded in a host that owns all device memory (a framework's caching
+ * allocator, a plugin interface that hands over only inputs and outputs) or latency-bound
+ * loops where cudaMalloc/cudaFree would synchronize the device.  The pages describe no
+ * such entry point; it exists only for such integrations.
+ * The window's k'/v' scratch is a fixed array of DP_NOALLOC_SCRATCH_BYTES inside the
+ * library's device memory, held by every device that loads the library until the process
+ * exits.  The call allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * CAPACITY, before anything is enqueued, if 2 * n_win * n_heads * head_dim feature
+ * elements (2 bytes each for bf16 windows, 4 for fp32) exceed that size.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress, with that device
+ * current); make that first call before any stream capture.  All calls share the one
+ * array: calls whose work overlaps on the GPU (other streams, other threads) race on it;
+ * order them on one stream.  Its contents from earlier calls are never read (the
+ * modulation prepass overwrites every element it uses).  Arguments, results and errors are
+ * otherwise those of dp_window_step. */
+dp_status dp_window_step_noalloc(const void* q, const void* k, const void* v, int64_t n_win,
+                                 const dp_blocks* blk, dp_kvcache* cache, const void* residual,
+                                 void* out, int32_t n_heads, int32_t head_dim, uint32_t flags,
+                                 dp_queue* queue, const void* push_noise, int64_t push_rows,
+                                 dp_dtype dt, void* stream);
+
 /* ---------------------------------------------------------------- profiling */
 
 /* Stage timing of dp_window_step.  After dp_profile_begin(max_steps), the next max_steps

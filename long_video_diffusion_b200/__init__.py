@@ -77,6 +77,8 @@ _SIGS = {
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
     "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
+    "dp_window_step_noalloc": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P,
+                               _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
     "dp_profile_begin": [_I32],
     "dp_profile_end": [ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_I32)],
     "dp_set_device": [_I32],
@@ -313,6 +315,31 @@ def profile_end():
     _check(_lib.dp_profile_end(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(n)),
            "dp_profile_end")
     return a.value, b.value, c.value, n.value
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def window_step_noalloc(q, k, v, blocks: DpBlocks, cache: KVCache, out, n_heads: int, head_dim: int,
+                        pop: bool = False, queue: Optional[Queue] = None, push_noise=None, push_rows=None,
+                        residual=None, stream=None, n_win: Optional[int] = None) -> None:
+    """window_step without kv_work, for callers that cannot allocate device memory: the
+    k'/v' scratch is a fixed NOALLOC_SCRATCH_BYTES array inside the library (see
+    dp_window_step_noalloc).  Calls share that array, so they must not overlap on the GPU."""
+    if isinstance(q, torch.Tensor):
+        ref = q
+        n = q.shape[0]
+        qp, kp, vp = _ptr(q), _ptr(k), _ptr(v)
+    else:
+        ref = out
+        n = int(n_win)
+        qp, kp, vp = ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v)
+    rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
+    _check(_lib.dp_window_step_noalloc(qp, kp, vp, n, ctypes.byref(blocks), ctypes.byref(cache.desc),
+                                       _ptr(residual), _ptr(out), n_heads, head_dim, STEP_POP if pop else 0,
+                                       ctypes.byref(queue.desc) if queue is not None else None,
+                                       _ptr(push_noise), int(rows), _dtype(out), _stream(ref, stream)),
+           "dp_window_step_noalloc")
 
 
 def device_status(stream=None) -> int:

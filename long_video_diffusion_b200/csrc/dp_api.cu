@@ -185,6 +185,10 @@ int32_t apply_push(dp_queue* q, int64_t rows) {
 
 }  // namespace
 
+namespace dp {
+dp_status set_error(dp_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace dp
+
 extern "C" {
 
 int32_t dp_version(void) { return 100; }

@@ -61,6 +61,9 @@ constexpr int kMaxCopySegs = 4;
 // Tensor-core path: q, residual, out bf16; k, v, cache f16 (f16_features) or bf16.
 cudaError_t launch_attention_tc(const AttnArgs& a, bool f16_features, cudaStream_t s);
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s);
+
+// Records `msg` as this thread's dp_last_error_detail() and returns `s` (dp_api.cu).
+dp_status set_error(dp_status s, const char* msg);
 // x_dt -> y_dt: bf16 -> bf16, bf16 -> f16 (saturating), f16 -> f16, f32 -> f32.
 cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, int64_t n_rows,
                             int hidden, const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s);
