@@ -58,6 +58,23 @@ static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "r
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
+// exp2 on the FMA pipe for part of the softmax (the MUFU unit retires 16 exp2 per clock per
+// SM, half the tensor-core rate at head_dim 64): 2^x = 2^n p(f), n = round(x) (added to the
+// exponent field), f = x - n in [-1/2, 1/2], p the degree-3 minimax polynomial of 2^f
+// (max relative error 7.5e-5, below f16's half ulp), coefficients from
+// csrc/fit_exp2_poly.py.  x >= -125 keeps the exponent field positive.
+constexpr float kPolyC0 = 0.9999280571937561f;
+constexpr float kPolyC1 = 0.6932609677314758f;
+constexpr float kPolyC2 = 0.2426111251115799f;
+constexpr float kPolyC3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer
+constexpr float kPolyMinX = -125.0f;
+// Column pairs (of the 16 in each 32-column chunk) whose exponentials use the polynomial.
+template <int HD>
+struct PolyPairs {
+  static constexpr uint32_t kMask = HD == 64 ? 0x4A52u : 0u;  // 6 of 16 at head_dim 64; none at 128
+};
+
 template <int HD>
 struct Layout {
   static constexpr int KCH = HD / 64;                    // 128-byte column chunks
@@ -103,9 +120,9 @@ struct Params {
 
 // Bounded wait that ignores the abort flag: used to drain work this CTA already issued.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
-  const uint64_t t0 = globaltimer();
+  const long long t0 = sm_clock();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (sm_clock() - t0 > kWaitLimitCycles) {
       atomicOr(status, DEV_ERR_TIMEOUT_DRAIN);
       return;
     }
@@ -146,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(v_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(kv_empty(s), NQ);  // one arrival from each query tile's PV issuer
     }
     for (int g = 0; g < NQ; ++g) {
       mbar_init(q_full(g), 128);
@@ -155,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full(g), 128);
       mbar_init(o_done(g), 1);
     }
-    mbar_init(fin, 1);
+    mbar_init(fin, 1 + NQ);     // one arrival from each MMA issuer
     *abort = 0;
     fence_mbar_init();
   }
@@ -205,79 +222,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(v_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    // Polls both query tiles' barriers and issues whichever product is ready, so neither
-    // softmax warpgroup waits for the other:
-    //   S_g(t) = Q_g K_t^T   needs K_t, and S_g(t-1) consumed (read by the softmax when P
-    //                        has its own columns; else PV_g(t-1) issued, since MMAs from
-    //                        this thread execute in issue order and P_g(t-1) lives in S_g)
-    //   O_g += P_g(t) V_t    needs P_g(t) and V_t
-    // The K/V stage of tile t is released once both query tiles' PV(t) are issued.
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_f32acc(Operand<F16>::kFmt, BM, BN, false);
-      constexpr uint32_t idPV = idesc_f32acc(Operand<F16>::kFmt, BM, HD, true);
-      auto issue_s = [&](int g, int st) {
-        const uint32_t qa = sb + L::OFF_Q + g * L::Q_BYTES;
-        const uint32_t ka = sb + L::OFF_K + st * L::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + g * BN, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int g, int st, bool acc) {
-        const uint32_t va = sb + L::OFF_V + st * L::KV_BYTES;
-        const uint32_t pa = tmem + L::COL_P + g * L::P_STRIDE;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tmem + L::COL_O + g * HD, pa + kk * 8, sdesc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), idPV,
-                 (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_full(0), 0, abort, p.status, DEV_ERR_TIMEOUT_Q) &&
-                mbar_wait(q_full(1), 0, abort, p.status, DEV_ERR_TIMEOUT_Q);
-      if (ok) tc_fence_after();
-      int ns[NQ] = {0, 0};  // next S tile per query tile
-      int np[NQ] = {0, 0};  // next PV tile per query tile
-      uint64_t t_last = globaltimer();
-      while (ok && (np[0] < n_tiles || np[1] < n_tiles)) {
-        bool progress = false;
-#pragma unroll
+  } else if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuers
+    // Three warps on three different SM sub-partitions issue the products, so that each
+    // gets its own share of issue slots next to the busy softmax warps there:
+    //   warp 9:  S_g(t) = Q_g K_t^T for both query tiles; needs K_t and S_g(t-1) consumed
+    //            (read by the softmax when P has its own columns; when P is written over
+    //            S_g, PV_g(t-1) complete);
+    //   warp 10 + g:  O_g += P_g(t) V_t; needs P_g(t) and V_t; releases the K/V stage
+    //            (kv_empty counts one arrival per query tile).
+    // Each issuer waits with bounded waits and commits its own products.
+    constexpr uint32_t idS = idesc_f32acc(Operand<F16>::kFmt, BM, BN, false);
+    constexpr uint32_t idPV = idesc_f32acc(Operand<F16>::kFmt, BM, HD, true);
+    // Descriptors are built once; each MMA adds a compile-time offset to the 14-bit start
+    // address field (16-byte units; every address stays below 2^18 bytes, so the sum never
+    // carries out of the field).
+    auto wait = [&](uint32_t bar, uint32_t parity, uint32_t code) {
+      return mbar_wait(bar, parity, abort, p.status, code);
+    };
+    bool ok = wait(q_full(0), 0, DEV_ERR_TIMEOUT_Q) && wait(q_full(1), 0, DEV_ERR_TIMEOUT_Q);
+    if (warp == 9) {
+      const uint64_t dq0 = sdesc_sw128(sb + L::OFF_Q, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sb + L::OFF_K, 16, 1024);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const int st = t % L::STAGES;
+        const uint64_t dk = dk0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
+#pragma unroll 1
         for (int g = 0; g < NQ; ++g) {
-          const int ts = ns[g];
-          if (ts < n_tiles) {
-            bool ready = ts == 0 || (L::SEP_P ? mbar_try_wait(s_free(g), (ts - 1) & 1) : np[g] >= ts);
-            ready = ready && mbar_try_wait(k_full(ts % L::STAGES), (ts / L::STAGES) & 1);
-            if (ready) {
-              tc_fence_after();
-              issue_s(g, ts % L::STAGES);
-              mma_commit(s_full(g));
-              ns[g] = ts + 1;
-              progress = true;
-            }
+          if (t > 0) {
+            ok = L::SEP_P ? wait(s_free(g), (t - 1) & 1, DEV_ERR_TIMEOUT_S)
+                          : wait(o_done(g), (t - 1) & 1, DEV_ERR_TIMEOUT_O);
+            if (!ok) break;
           }
-          const int tp = np[g];
-          if (tp < ns[g] && mbar_try_wait(p_full(g), tp & 1) &&
-              mbar_try_wait(v_full(tp % L::STAGES), (tp / L::STAGES) & 1)) {
-            tc_fence_after();
-            issue_pv(g, tp % L::STAGES, tp > 0);
-            mma_commit(o_done(g));
-            np[g] = tp + 1;
-            if (np[1 - g] > tp) mma_commit(kv_empty(tp % L::STAGES));
-            progress = true;
+          if (g == 0) {
+            ok = wait(k_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
+            if (!ok) break;
           }
-        }
-        if (progress) {
-          t_last = globaltimer();
-        } else if (*abort) {
-          break;
-        } else if (globaltimer() - t_last > kWaitLimitNs) {
-          atomicOr(p.status, DEV_ERR_TIMEOUT_P);
-          *abort = 1;
-          break;
+          tc_fence_after();
+          const uint64_t dq = dq0 + static_cast<uint64_t>((g * L::Q_BYTES) >> 4);
+          const uint32_t d = tmem + g * BN;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32) >> 4);
+            mma_ss(d, dq + off, dk + off, idS, kk > 0);
+          }
+          mma_commit(s_full(g));
         }
       }
+    } else if (warp == 10 || warp == 11) {
+      const int g = warp - 10;
+      const uint64_t dv0 = sdesc_sw128(sb + L::OFF_V, L::CHUNK_BYTES, 1024);
+      const uint32_t pa = tmem + L::COL_P + g * L::P_STRIDE;
+      const uint32_t d = tmem + L::COL_O + g * HD;
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const int st = t % L::STAGES;
+        ok = wait(p_full(g), t & 1, DEV_ERR_TIMEOUT_P) && wait(v_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d, pa + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idPV, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(o_done(g));
+        mma_commit(kv_empty(st));
+      }
+    }
+    if (warp >= 9) {
+      // every product this warp issued completes before TMEM is released
       mma_commit(fin);
       drain_wait(fin, 0, p.status);
     }
@@ -362,30 +373,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c)
             if (i * 32 + c >= valid) sr[i][c] = 0xff800000u;
       }
-      // row max: four independent chains of 3-input max
-      float mc[4];
+      // row max: eight independent chains of 3-input max (short dependency chains)
+      float mc[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float m = fmaxf(__uint_as_float(sr[i][0]), __uint_as_float(sr[i][31]));
+      for (int h = 0; h < 8; ++h) {
+        const uint32_t* r = &sr[h >> 1][(h & 1) * 16];
+        float m = fmaxf(__uint_as_float(r[0]), __uint_as_float(r[15]));
 #pragma unroll
-        for (int c = 1; c < 31; c += 2) m = fmax3(m, __uint_as_float(sr[i][c]), __uint_as_float(sr[i][c + 1]));
-        mc[i] = m;
+        for (int c = 1; c < 15; c += 2) m = fmax3(m, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        mc[h] = m;
       }
-      const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]);
+      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
       const float m_new = fmaxf(m_ref, mx * p.scale_log2);
       if (j == 0) {
         m_ref = m_new;
       } else {
         const bool need = m_new > m_ref + kRescaleLog2;
         const bool any_need = __any_sync(0xffffffffu, need);
-        if (L::SEP_P || any_need) {
-          // PV(j-1) must be complete before O is rescaled or P(j-1) is overwritten
+        if (any_need) {
+          // PV(j-1) must be complete before O is rescaled
           ok = mbar_wait(o_done(g), (j - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-        }
-        if (any_need) {
           const float f = need ? ex2_approx(m_ref - m_new) : 1.0f;
 #pragma unroll
           for (int c0 = 0; c0 < HD; c0 += 32) {
@@ -403,28 +413,59 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // P = exp2(s * scale * log2(e) - m_ref): packed FMA, MUFU exp2, packed adds
+      // P = exp2(s * scale * log2(e) - m_ref): packed FMA, exp2 on the MUFU unit or (for
+      // the PolyPairs columns) on the FMA pipe, packed adds for the row sum
       const uint64_t nm2 = f32x2(-m_ref, -m_ref);
+      const uint64_t magic2 = f32x2(kRoundMagic, kRoundMagic);
+      const uint64_t nmagic2 = f32x2(-kRoundMagic, -kRoundMagic);
+      const uint64_t neg1_2 = f32x2(-1.0f, -1.0f);
+      const uint64_t c0_2 = f32x2(kPolyC0, kPolyC0), c1_2 = f32x2(kPolyC1, kPolyC1);
+      const uint64_t c2_2 = f32x2(kPolyC2, kPolyC2), c3_2 = f32x2(kPolyC3, kPolyC3);
       uint64_t acc0 = f32x2(0.0f, 0.0f), acc1 = acc0;
+      uint32_t pk[4][16];  // P stays in registers until PV(j-1) has released its columns
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint64_t x = ffma2(f32x2(__uint_as_float(sr[i][2 * c]), __uint_as_float(sr[i][2 * c + 1])), sl2, nm2);
           float x0, x1;
           f32x2_split(x, x0, x1);
-          const float a = ex2_approx(x0);
-          const float b = ex2_approx(x1);
+          float a, b;
+          if ((PolyPairs<HD>::kMask >> c) & 1u) {
+            const uint64_t xc = f32x2(fmaxf(x0, kPolyMinX), fmaxf(x1, kPolyMinX));
+            const uint64_t t = fadd2(xc, magic2);        // low mantissa bits hold round(x)
+            const uint64_t f = ffma2(fadd2(t, nmagic2), neg1_2, xc);  // x - round(x)
+            uint64_t q = ffma2(c3_2, f, c2_2);
+            q = ffma2(q, f, c1_2);
+            q = ffma2(q, f, c0_2);
+            float q0, q1, t0, t1;
+            f32x2_split(q, q0, q1);
+            f32x2_split(t, t0, t1);
+            a = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+            b = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+          } else {
+            a = ex2_approx(x0);
+            b = ex2_approx(x1);
+          }
           const uint64_t ab = f32x2(a, b);
           if (c & 1)
             acc1 = fadd2(acc1, ab);
           else
             acc0 = fadd2(acc0, ab);
-          pk[c] = Operand<F16>::pack_p(a, b);
+          pk[i][c] = Operand<F16>::pack_p(a, b);
         }
-        tmem_st16(trow + p_col + i * 16, pk);
       }
+      if constexpr (L::SEP_P) {
+        if (j > 0) {
+          // P(j-1) in these columns must have been read by PV(j-1); by now it has been
+          ok = mbar_wait(o_done(g), (j - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_st16(trow + p_col + i * 16, pk[i]);
       {
         const uint64_t acc = fadd2(acc0, acc1);
         float a0, a1;

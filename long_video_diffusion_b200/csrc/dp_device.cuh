@@ -20,18 +20,16 @@ enum : uint32_t {
   DEV_ERR_TIMEOUT_DRAIN = 1u << 6,
 };
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;
+// A bounded wait gives up after this many SM clock cycles (about 2 s at 2 GHz, longer at
+// lower clocks).  The SM cycle counter is cheap to read; the global nanosecond timer is
+// not, and reading it inside a polling loop delays the loop by hundreds of cycles.
+constexpr long long kWaitLimitCycles = 4000ll * 1000ll * 1000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
+__device__ __forceinline__ long long sm_clock() { return clock64(); }
 
 __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
@@ -70,20 +68,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition (for polling several barriers: try_wait may
+// suspend the thread for an implementation-defined time before reporting "not yet").
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
-// kWaitLimitNs, or as soon as *abort (shared) is set by another role: on giving up it
+// kWaitLimitCycles, or as soon as *abort (shared) is set by another role: on giving up it
 // records `code` in the device status word, raises *abort and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint32_t code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
+  // test_wait first: a completed phase is reported at once (try_wait is slow to return
+  // even then); try_wait, which can suspend the thread, only while the phase is pending
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = sm_clock();
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      atomicOr(status, code);
-      *abort = 1;
-      return false;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (sm_clock() - t0 > kWaitLimitCycles) {
+        atomicOr(status, code);
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
