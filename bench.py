@@ -29,7 +29,24 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 1 B200"
+
+# DRAM bytes (read + write) of one attention launch from an ncu capture (summaries under
+# profiles/), valid only for the kernel source they were captured on (md5 of
+# csrc/dp_attn_tc.cu); any other source reports null.
+TRAFFIC_SOURCE_MD5 = "4640b0b89f56c60bf7430dd4a1674f0a"
+TRAFFIC_BYTES = {"cogvideo_bf16": 232.817152e6 + 53.842432e6, "wan_bf16": 603.7056e6 + 141.67936e6}
 L2_BYTES = 126 * 1024 * 1024
+
+
+def attention_traffic(config_name: str):
+    import hashlib
+    path = os.path.join(ROOT, "long_video_diffusion_b200", "csrc", "dp_attn_tc.cu")
+    try:
+        with open(path, "rb") as f:
+            md5 = hashlib.md5(f.read()).hexdigest()
+    except OSError:
+        return None
+    return TRAFFIC_BYTES.get(config_name) if md5 == TRAFFIC_SOURCE_MD5 else None
 
 
 def load_peaks():
@@ -387,7 +404,9 @@ def main():
             "attn_tflops": achieved,
             "stage_ms": {"modulate": r["mod_ms"], "attention": r["attn_ms"], "advance": r["adv_ms"]},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "window_attn_tc_kernel",
+                         "frac": achieved / peak, "traffic": attention_traffic(args.config),
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                         "kernel": "window_attn_tc_kernel",
                          "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
                          "algorithmic_flop_per_launch": flop},
             "stage_hbm": stage_hbm(cfg, r, peaks),
