@@ -64,6 +64,12 @@ typedef enum { DP_F32 = 0, DP_BF16 = 1, DP_F16 = 2 } dp_dtype;
 /* dp_window_attention flags */
 #define DP_MOD_Q 1u     /* prologue: q' = q * (1 + scale_b) + shift_b, b = block of the row */
 #define DP_GATE_OUT 2u  /* epilogue: out = gate_b * o (+ residual) */
+/* Test hook for the failure path of the tensor-core kernel: its producer issues no K/V
+ * loads, so every wait for them gives up at its bound (about 2 s of SM clock); the kernel
+ * then stops, releases its resources and returns without writing `out`, and
+ * dp_device_status() reports DP_ERR_TIMEOUT.  Nothing faults or hangs.  Use it with a
+ * small launch (one CTA: n_win <= 256 rows and one head) so that one bound elapses. */
+#define DP_TEST_SKIP_KV_LOADS 0x80000000u
 
 /* dp_window_step flags */
 #define DP_STEP_POP 1u  /* after attention, the head block exits: its K'/V' rows become the

@@ -30,6 +30,7 @@ MAX_SLOTS = 16
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_CAPACITY, ERR_TIMEOUT, ERR_EMPTY = 0, -1, -2, -3, -4, -5, -6
 F32, BF16, F16 = 0, 1, 2
 MOD_Q, GATE_OUT = 1, 2
+TEST_SKIP_KV_LOADS = 0x80000000
 STEP_POP = 1
 
 if not os.path.exists(LIB_PATH):

@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      const bool skip_loads = (p.flags & DP_TEST_SKIP_KV_LOADS) != 0;  // failure-path test hook
+      for (int j = 0; j < n_tiles && !skip_loads; ++j) {
         const int st = j % L::STAGES;
         const int use = j / L::STAGES;
         if (use > 0 && !mbar_wait(kv_empty(st), (use - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_EMPTY)) break;
