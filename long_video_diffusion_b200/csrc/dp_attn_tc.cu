@@ -16,16 +16,19 @@
 //   warps 0-3  softmax warpgroup for query tile 0 (one thread per query row)
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp 8     TMA producer: K and V tiles into a ring of shared-memory stages
-//   warp 9     TMEM owner and MMA issuer (one thread issues tcgen05.mma)
-//   warps 10-11 idle (they complete the third warpgroup, which setmaxnreg needs)
-// Registers: launched at kLaunchRegs per thread; the producer warpgroup gives registers
-// back (kLowRegs) and the two softmax warpgroups take them (kHighRegs), so a softmax
-// thread can hold its 128 scores without spilling.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+HD), O1 after it.
-// P (bf16) is written over the first 64 columns of its S tile and consumed from TMEM as
-// the A operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both
-// K-major with the 128-byte swizzle; V is the MN-major B operand of the PV product.
-// Softmax is fp32 with exp2 on the MUFU unit; the running max is only moved (and O
+//   warp 9     TMEM owner; issues S_g = Q_g K^T for both query tiles
+//   warps 10-11 issue O_g += P_g V, one warp per query tile (three issuing warps on three
+//              SM sub-partitions, so no single warp's issue slots serialise the products)
+// Registers: launched at kLaunchRegs per thread; the producer/issuer warpgroup gives
+// registers back (kLowRegs) and the two softmax warpgroups take them (kHighRegs), so a
+// softmax thread can hold its 128 scores without spilling.
+// Tensor memory (512 columns): S0, S1 (128 fp32 columns each), O0, O1 (HD columns each) and,
+// when there is room (head_dim 64), P0, P1 in their own 64 columns; otherwise P is written
+// over the first 64 columns of its S tile.  P (16-bit pairs) is consumed from TMEM as the A
+// operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both K-major with
+// the 128-byte swizzle; V is the MN-major B operand of the PV product.
+// Softmax is fp32 with exp2 on the MUFU unit (part of it on the FMA pipe at head_dim 64,
+// see PolyPairs); the running max is only moved (and O
 // rescaled) when it grows by more than 2^8, which keeps the result exact because the
 // final 1/l uses the same reference max as the numerator.
 // Every wait is bounded (see dp_device.cuh): on giving up the kernel records a timeout in
