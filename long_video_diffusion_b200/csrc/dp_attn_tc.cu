@@ -12,20 +12,22 @@
 // significand: rounding the modulated features to bf16 alone costs about 2.5e-2 absolute on
 // peaked softmaxes, f16 about 3e-3) or bf16; both accumulate in fp32.
 //
-// Design (one CTA = two 128-row query tiles of one head; keys in 128-row tiles):
+// Design (one CTA = two 128-row query tiles of one head; keys in tiles of BN rows, 128 at
+// head_dim 64 and 64 at head_dim 128):
 //   warps 0-3  softmax warpgroup for query tile 0 (one thread per query row)
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp 8     TMA producer: K and V tiles into a ring of shared-memory stages
-//   warp 9     TMEM owner; issues S_g = Q_g K^T for both query tiles
-//   warps 10-11 issue O_g += P_g V, one warp per query tile (three issuing warps on three
-//              SM sub-partitions, so no single warp's issue slots serialise the products)
+//   warps 9-11 issue the products S_g = Q_g K^T and O_g += P_g V, split so that each warp
+//              issues the same number per key tile (head_dim 64: warp 9 S for both query
+//              tiles, warps 10-11 PV per tile; head_dim 128: warps 9-10 S per tile, warp 11
+//              PV for both); warp 9 also owns the tensor memory
 // Registers: launched at kLaunchRegs per thread; the producer/issuer warpgroup gives
 // registers back (kLowRegs) and the two softmax warpgroups take them (kHighRegs), so a
-// softmax thread can hold its 128 scores without spilling.
-// Tensor memory (512 columns): S0, S1 (128 fp32 columns each), O0, O1 (HD columns each) and,
-// when there is room (head_dim 64), P0, P1 in their own 64 columns; otherwise P is written
-// over the first 64 columns of its S tile.  P (16-bit pairs) is consumed from TMEM as the A
-// operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both K-major with
+// softmax thread can hold its scores without spilling.
+// Tensor memory (512 columns): S0, S1 (BN fp32 columns each), O0, O1 (HD columns each) and
+// P0, P1 (BN/2 columns each); with these tile widths P always has columns of its own, so the
+// next S product runs while the softmax still works on the current tile.  P (16-bit pairs)
+// is consumed from TMEM as the A operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both K-major with
 // the 128-byte swizzle; V is the MN-major B operand of the PV product.
 // Softmax is fp32 with exp2 on the MUFU unit (part of it on the FMA pipe at head_dim 64,
 // see PolyPairs); the running max is only moved (and O
@@ -51,7 +53,6 @@ namespace dp {
 namespace {
 
 constexpr int BM = 128;       // query rows per tile
-constexpr int BN = 128;       // keys per tile
 constexpr int NQ = 2;         // query tiles per CTA
 constexpr int kThreads = 384; // 12 warps
 constexpr int kLaunchRegs = 168;  // 65536 / 384 rounded down to the allocation granule
@@ -80,19 +81,34 @@ struct PolyPairs {
 
 template <int HD>
 struct Layout {
+  // Keys per tile: 128 at head_dim 64; 64 at head_dim 128, so that P gets tensor-memory
+  // columns of its own there too (see below).  A 128x64x16 product costs about 3/4 of a
+  // 128x128x16 one on the tensor pipe, a smaller price than running each query tile's
+  // S -> softmax -> PV -> S chain strictly in series.
+  static constexpr int BN = HD == 64 ? 128 : 64;
   static constexpr int KCH = HD / 64;                    // 128-byte column chunks
-  static constexpr int STAGES = (HD == 64) ? 4 : 2;
-  static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 B
+  static constexpr int STAGES = 4;
+  static constexpr int Q_CHUNK = BM * 128;               // one 64-column chunk of a Q tile
+  static constexpr int KV_CHUNK = BN * 128;              // one 64-column chunk of a K or V tile
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   // Tensor memory: S_g (BN fp32 columns each), P_g (BN/2 columns of 16-bit pairs), O_g (HD
   // columns).  When all of it fits, P has its own columns and the next S product can run
   // while the softmax still works on the current tile; otherwise P is written over S_g.
-  static constexpr bool SEP_P = 2 * BN + 2 * (BN / 2) + 2 * HD <= kTmemCols;
-  static constexpr int COL_P = SEP_P ? 2 * BN : 0;
+  // The wider of the S and O regions comes first, so every region starts at a multiple of
+  // its own width.
+  static constexpr bool SEP_P = NQ * BN + NQ * (BN / 2) + NQ * HD <= kTmemCols;
+  static constexpr bool O_FIRST = HD > BN;
+  static constexpr int COL_S = O_FIRST ? NQ * HD : 0;
+  static constexpr int COL_P = SEP_P ? COL_S + NQ * BN : COL_S;
   static constexpr int P_STRIDE = SEP_P ? BN / 2 : BN;
-  static constexpr int COL_O = SEP_P ? 3 * BN : 2 * BN;
-  static_assert(COL_O + NQ * HD <= kTmemCols, "tensor memory budget");
+  static constexpr int COL_O = O_FIRST ? 0 : (SEP_P ? COL_P + NQ * (BN / 2) : NQ * BN);
+  static_assert(BN % 32 == 0 && (BN / 16 == 4 || BN / 16 == 8), "key tile width");
+  // Issue split (see the MMA issuers): one warp per query tile issues S when S has more
+  // products per key tile than PV (HD / 16 against BN / 16), else one warp per query tile
+  // issues PV.
+  static constexpr bool S_PER_G = HD > BN;
+  static_assert((O_FIRST ? COL_P + NQ * P_STRIDE : COL_O + NQ * HD) <= kTmemCols, "tensor memory budget");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
@@ -140,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
                           const Params p) {
   using L = Layout<HD>;
+  constexpr int BN = L::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -166,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(v_full(s), 1);
-      mbar_init(kv_empty(s), NQ);  // one arrival from each query tile's PV issuer
+      mbar_init(kv_empty(s), L::S_PER_G ? 1 : NQ);  // one arrival from each PV issuing warp
     }
     for (int g = 0; g < NQ; ++g) {
       mbar_init(q_full(g), 128);
@@ -212,11 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(k_full(st), L::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < L::KCH; ++c)
-          tma_load_2d(sb + L::OFF_K + st * L::KV_BYTES + c * L::CHUNK_BYTES, mk, head * HD + c * 64, row, k_full(st));
+          tma_load_2d(sb + L::OFF_K + st * L::KV_BYTES + c * L::KV_CHUNK, mk, head * HD + c * 64, row, k_full(st));
         mbar_arrive_expect_tx(v_full(st), L::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < L::KCH; ++c)
-          tma_load_2d(sb + L::OFF_V + st * L::KV_BYTES + c * L::CHUNK_BYTES, mv, head * HD + c * 64, row, v_full(st));
+          tma_load_2d(sb + L::OFF_V + st * L::KV_BYTES + c * L::KV_CHUNK, mv, head * HD + c * 64, row, v_full(st));
         issued = j + 1;
       }
       // every copy this CTA issued must land before its shared memory is released
@@ -228,67 +245,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issuers
-    // Three warps on three different SM sub-partitions issue the products, so that each
-    // gets its own share of issue slots next to the busy softmax warps there:
-    //   warp 9:  S_g(t) = Q_g K_t^T for both query tiles; needs K_t and S_g(t-1) consumed
-    //            (read by the softmax when P has its own columns; when P is written over
-    //            S_g, PV_g(t-1) complete);
-    //   warp 10 + g:  O_g += P_g(t) V_t; needs P_g(t) and V_t; releases the K/V stage
-    //            (kv_empty counts one arrival per query tile).
+    // Products: S_g(t) = Q_g K_t^T needs K_t and S_g(t-1) consumed (read by the softmax when
+    // P has its own columns; PV_g(t-1) complete when P is written over S_g); O_g += P_g(t) V_t
+    // needs P_g(t) and V_t and releases the K/V stage.  A tcgen05.mma holds its issuing
+    // thread while the tensor pipe's queue is full, so a warp's barrier tests and commits run
+    // in series with the execution of its own products.  Three warps on three SM
+    // sub-partitions therefore share the issuing, split so that each issues the same number
+    // of products per key tile:
+    //   head_dim 64 (4 S and 8 PV products per query tile): warp 9 S for both query
+    //     tiles, warp 10 + g PV_g;
+    //   head_dim 128 (8 S and 4 PV products per query tile): warp 9 + g S_g, warp 11 PV
+    //     for both query tiles.
     // Each issuer waits with bounded waits and commits its own products.
     constexpr uint32_t idS = idesc_f32acc(Operand<F16>::kFmt, BM, BN, false);
     constexpr uint32_t idPV = idesc_f32acc(Operand<F16>::kFmt, BM, HD, true);
-    // Descriptors are built once; each MMA adds a compile-time offset to the 14-bit start
-    // address field (16-byte units; every address stays below 2^18 bytes, so the sum never
-    // carries out of the field).
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t code) {
       return mbar_wait(bar, parity, abort, p.status, code);
     };
+    // two waits with one overlapped fast path
+    auto wait2 = [&](uint32_t b0, uint32_t p0, uint32_t c0, uint32_t b1, uint32_t p1, uint32_t c1) {
+      return mbar_test_wait2(b0, p0, b1, p1) || (wait(b0, p0, c0) && wait(b1, p1, c1));
+    };
+    // Descriptors are built once; each MMA adds a compile-time offset to the 14-bit start
+    // address field (16-byte units; every address stays below 2^18 bytes, so the sum never
+    // carries out of the field).
+    const uint64_t dq0 = sdesc_sw128(sb + L::OFF_Q, 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(sb + L::OFF_K, 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(sb + L::OFF_V, L::KV_CHUNK, 1024);
     bool ok = wait(q_full(0), 0, DEV_ERR_TIMEOUT_Q) && wait(q_full(1), 0, DEV_ERR_TIMEOUT_Q);
-    if (warp == 9) {
-      const uint64_t dq0 = sdesc_sw128(sb + L::OFF_Q, 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(sb + L::OFF_K, 16, 1024);
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        const int st = t % L::STAGES;
-        const uint64_t dk = dk0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
-#pragma unroll 1
-        for (int g = 0; g < NQ; ++g) {
-          if (t > 0) {
-            ok = L::SEP_P ? wait(s_free(g), (t - 1) & 1, DEV_ERR_TIMEOUT_S)
-                          : wait(o_done(g), (t - 1) & 1, DEV_ERR_TIMEOUT_O);
-            if (!ok) break;
-          }
-          if (g == 0) {
-            ok = wait(k_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
-            if (!ok) break;
-          }
-          tc_fence_after();
-          const uint64_t dq = dq0 + static_cast<uint64_t>((g * L::Q_BYTES) >> 4);
-          const uint32_t d = tmem + g * BN;
+    // S_g(t) into S_g's columns (the caller has waited for K_t and for S_g(t-1) to be free)
+    auto mma_s = [&](int st, int g) {
+      tc_fence_after();
+      const uint64_t dq = dq0 + static_cast<uint64_t>((g * L::Q_BYTES) >> 4);
+      const uint64_t dk = dk0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
+      const uint32_t d = tmem + L::COL_S + g * BN;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32) >> 4);
-            mma_ss(d, dq + off, dk + off, idS, kk > 0);
-          }
-          mma_commit(s_full(g));
-        }
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t oq = static_cast<uint64_t>(((kk >> 2) * L::Q_CHUNK + (kk & 3) * 32) >> 4);
+        const uint64_t okv = static_cast<uint64_t>(((kk >> 2) * L::KV_CHUNK + (kk & 3) * 32) >> 4);
+        mma_ss(d, dq + oq, dk + okv, idS, kk > 0);
       }
-    } else if (warp == 10 || warp == 11) {
-      const int g = warp - 10;
-      const uint64_t dv0 = sdesc_sw128(sb + L::OFF_V, L::CHUNK_BYTES, 1024);
+      mma_commit(s_full(g));
+    };
+    // O_g += P_g(t) V_t (the caller has waited for P_g(t) and V_t)
+    auto mma_pv = [&](int t, int st, int g) {
+      tc_fence_after();
+      const uint64_t dv = dv0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
       const uint32_t pa = tmem + L::COL_P + g * L::P_STRIDE;
       const uint32_t d = tmem + L::COL_O + g * HD;
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        const int st = t % L::STAGES;
-        ok = wait(p_full(g), t & 1, DEV_ERR_TIMEOUT_P) && wait(v_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t dv = dv0 + static_cast<uint64_t>((st * L::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d, pa + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idPV, (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(o_done(g));
-        mma_commit(kv_empty(st));
+      for (int kk = 0; kk < BN / 16; ++kk)
+        mma_ts(d, pa + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idPV, (t > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(o_done(g));
+    };
+    if constexpr (L::S_PER_G) {
+      if (warp == 9 || warp == 10) {
+        const int g = warp - 9;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const int st = t % L::STAGES;
+          const uint32_t kpar = (t / L::STAGES) & 1;
+          // both phases have normally completed: one overlapped test usually settles it
+          if (t > 0)
+            ok = wait2(L::SEP_P ? s_free(g) : o_done(g), (t - 1) & 1, L::SEP_P ? DEV_ERR_TIMEOUT_S : DEV_ERR_TIMEOUT_O,
+                       k_full(st), kpar, DEV_ERR_TIMEOUT_KV);
+          else
+            ok = wait(k_full(st), kpar, DEV_ERR_TIMEOUT_KV);
+          if (!ok) break;
+          mma_s(st, g);
+        }
+      } else if (warp == 11) {
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const int st = t % L::STAGES;
+#pragma unroll 1
+          for (int g = 0; g < NQ; ++g) {
+            ok = wait(p_full(g), t & 1, DEV_ERR_TIMEOUT_P) &&
+                 (g > 0 || wait(v_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV));
+            if (!ok) break;
+            mma_pv(t, st, g);
+          }
+          if (ok) mma_commit(kv_empty(st));  // after the stage's last PV product
+        }
+      }
+    } else {
+      if (warp == 9) {
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const int st = t % L::STAGES;
+#pragma unroll 1
+          for (int g = 0; g < NQ; ++g) {
+            if (t > 0) {
+              ok = L::SEP_P ? wait(s_free(g), (t - 1) & 1, DEV_ERR_TIMEOUT_S)
+                            : wait(o_done(g), (t - 1) & 1, DEV_ERR_TIMEOUT_O);
+              if (!ok) break;
+            }
+            if (g == 0) {
+              ok = wait(k_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
+              if (!ok) break;
+            }
+            mma_s(st, g);
+          }
+        }
+      } else if (warp == 10 || warp == 11) {
+        const int g = warp - 10;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const int st = t % L::STAGES;
+          ok = wait(p_full(g), t & 1, DEV_ERR_TIMEOUT_P) && wait(v_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
+          if (!ok) break;
+          mma_pv(t, st, g);
+          mma_commit(kv_empty(st));
+        }
       }
     }
     if (warp >= 9) {
@@ -338,14 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             Operand<F16>::pack(xf[4], xf[5]), Operand<F16>::pack(xf[6], xf[7]));
         }
         const int chunk = c >> 3, w = c & 7;
-        *reinterpret_cast<uint4*>(sq + chunk * L::CHUNK_BYTES + t * 128 + ((w ^ (t & 7)) << 4)) = outv;
+        *reinterpret_cast<uint4*>(sq + chunk * L::Q_CHUNK + t * 128 + ((w ^ (t & 7)) << 4)) = outv;
       }
       fence_proxy_async_smem();
       mbar_arrive(q_full(g));
     }
 
     const uint32_t trow = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
-    const uint32_t s_col = g * BN;
+    const uint32_t s_col = L::COL_S + g * BN;
+    constexpr int NCH = BN / 32;  // 32-column chunks of an S row
+    constexpr int NG = BN / 16;   // max chains
     const uint32_t p_col = L::COL_P + g * L::P_STRIDE;
     const uint32_t o_col = L::COL_O + g * HD;
     const uint64_t sl2 = f32x2(p.scale_log2, p.scale_log2);
@@ -358,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[NCH][32];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld32(trow + s_col + i * 32, sr[i]);
+      for (int i = 0; i < NCH; ++i) tmem_ld32(trow + s_col + i * 32, sr[i]);
       tmem_wait_ld();
       if constexpr (L::SEP_P) {
         // S is in registers: the tensor core may overwrite it with the next tile's S
@@ -372,22 +438,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (rem < BN) {  // last tile of a segment: keys beyond it get -inf (TMA filled them with 0)
         const int valid = static_cast<int>(rem);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < NCH; ++i)
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (i * 32 + c >= valid) sr[i][c] = 0xff800000u;
       }
-      // row max: eight independent chains of 3-input max (short dependency chains)
-      float mc[8];
+      // row max: NG independent chains of 3-input max (short dependency chains)
+      float mc[NG];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
+      for (int h = 0; h < NG; ++h) {
         const uint32_t* r = &sr[h >> 1][(h & 1) * 16];
         float m = fmaxf(__uint_as_float(r[0]), __uint_as_float(r[15]));
 #pragma unroll
         for (int c = 1; c < 15; c += 2) m = fmax3(m, __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
         mc[h] = m;
       }
-      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+      float mx;
+      if constexpr (NG == 8)
+        mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+      else
+        mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
       const float m_new = fmaxf(m_ref, mx * p.scale_log2);
       if (j == 0) {
         m_ref = m_new;
@@ -426,9 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t c0_2 = f32x2(kPolyC0, kPolyC0), c1_2 = f32x2(kPolyC1, kPolyC1);
       const uint64_t c2_2 = f32x2(kPolyC2, kPolyC2), c3_2 = f32x2(kPolyC3, kPolyC3);
       uint64_t acc0 = f32x2(0.0f, 0.0f), acc1 = acc0;
-      uint32_t pk[4][16];  // P stays in registers until PV(j-1) has released its columns
+      uint32_t pk[NCH][16];  // P stays in registers until PV(j-1) has released its columns
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < NCH; ++i) {
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint64_t x = ffma2(f32x2(__uint_as_float(sr[i][2 * c]), __uint_as_float(sr[i][2 * c + 1])), sl2, nm2);
@@ -469,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_st16(trow + p_col + i * 16, pk[i]);
+      for (int i = 0; i < NCH; ++i) tmem_st16(trow + p_col + i * 16, pk[i]);
       {
         const uint64_t acc = fadd2(acc0, acc1);
         float a0, a1;
@@ -560,11 +630,12 @@ template <int HD, bool F16>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   using L = Layout<HD>;
   CUtensorMap tkc, tvc, tkw, tvw;
-  if (!encode_tmap_16(&tkw, a.k, a.n_win, a.hidden, F16) || !encode_tmap_16(&tvw, a.v, a.n_win, a.hidden, F16))
+  constexpr int BN = L::BN;
+  if (!encode_tmap_16(&tkw, a.k, a.n_win, a.hidden, BN, F16) || !encode_tmap_16(&tvw, a.v, a.n_win, a.hidden, BN, F16))
     return cudaErrorInvalidValue;
   if (a.cache_len > 0) {
-    if (!encode_tmap_16(&tkc, a.cache_k, a.cache_len, a.hidden, F16) ||
-        !encode_tmap_16(&tvc, a.cache_v, a.cache_len, a.hidden, F16))
+    if (!encode_tmap_16(&tkc, a.cache_k, a.cache_len, a.hidden, BN, F16) ||
+        !encode_tmap_16(&tvc, a.cache_v, a.cache_len, a.hidden, BN, F16))
       return cudaErrorInvalidValue;
   } else {
     tkc = tkw;
@@ -607,12 +678,12 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, bool f16) {
+bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, int box_rows, bool f16) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(hidden) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(static_cast<CUtensorMap*>(tmap), f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

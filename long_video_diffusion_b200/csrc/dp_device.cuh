@@ -82,6 +82,22 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Both phases complete?  The two tests are issued before either result is used, so their
+// shared-memory round trips overlap.
+__device__ __forceinline__ bool mbar_test_wait2(uint32_t bar0, uint32_t par0, uint32_t bar1, uint32_t par1) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p1, [%3], %4;\n\t"
+      "and.pred p0, p0, p1;\n\t"
+      "selp.u32 %0, 1, 0, p0;\n\t}"
+      : "=r"(ok)
+      : "r"(bar0), "r"(par0), "r"(bar1), "r"(par1)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // kWaitLimitCycles, or as soon as *abort (shared) is set by another role: on giving up it
 // records `code` in the device status word, raises *abort and returns false.
@@ -234,6 +250,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
   return d;
+}
+
+// Descriptor d with its start address advanced by off16 16-byte units.  The start address
+// is the low 14 bits of the low word; callers keep every address below 2^18 bytes, so the
+// sum stays inside the field and only the low 32-bit word changes (an immediate add).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t off16) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(d));
+  lo += off16;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator (bit 4), A and B of one 16-bit type

@@ -70,7 +70,7 @@ cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, 
 cudaError_t launch_copy(const CopySeg* segs, int nseg, cudaStream_t s);
 
 // Host-side helper: encode a 2-D 16-bit (f16 or bf16) tensor map [rows][hidden] with a
-// {64, 128} box and 128-byte swizzle (defined in dp_attn_tc.cu).
-bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, bool f16);
+// {64 columns, box_rows rows} box and 128-byte swizzle (defined in dp_attn_tc.cu).
+bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, int box_rows, bool f16);
 
 }  // namespace dp
