@@ -29,7 +29,7 @@
 // next S product runs while the softmax still works on the current tile.  P (16-bit pairs)
 // is consumed from TMEM as the A operand of O += P V.  S = Q K^T uses Q and K tiles from shared memory, both K-major with
 // the 128-byte swizzle; V is the MN-major B operand of the PV product.
-// Softmax is fp32 with exp2 on the MUFU unit (part of it on the FMA pipe at head_dim 64,
+// Softmax is fp32 with exp2 on the MUFU unit (part of it on the FMA pipe,
 // see PolyPairs); the running max is only moved (and O
 // rescaled) when it grows by more than 2^8, which keeps the result exact because the
 // final 1/l uses the same reference max as the numerator.
@@ -63,7 +63,7 @@ constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
 // exp2 on the FMA pipe for part of the softmax (the MUFU unit retires 16 exp2 per clock per
-// SM, half the tensor-core rate at head_dim 64): 2^x = 2^n p(f), n = round(x) (added to the
+// SM, no more than the tensor cores need at either head dim): 2^x = 2^n p(f), n = round(x) (added to the
 // exponent field), f = x - n in [-1/2, 1/2], p the degree-3 minimax polynomial of 2^f
 // (max relative error 7.5e-5, below f16's half ulp), coefficients from
 // csrc/fit_exp2_poly.py.  x >= -125 keeps the exponent field positive.
@@ -73,10 +73,12 @@ constexpr float kPolyC2 = 0.2426111251115799f;
 constexpr float kPolyC3 = 0.0551716685295105f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer
 constexpr float kPolyMinX = -125.0f;
-// Column pairs (of the 16 in each 32-column chunk) whose exponentials use the polynomial.
+// Column pairs (of the 16 in each 32-column chunk) whose exponentials use the polynomial:
+// 6 of 16 (measured best at both head dims among 0, 3, 6, 8, 10 and 12 of 16; more moves
+// the limit to the FMA pipe, which the polynomial costs about seven instructions a pair).
 template <int HD>
 struct PolyPairs {
-  static constexpr uint32_t kMask = HD == 64 ? 0x4A52u : 0u;  // 6 of 16 at head_dim 64; none at 128
+  static constexpr uint32_t kMask = 0x4A52u;
 };
 
 template <int HD>
