@@ -31,22 +31,23 @@ if ROOT not in sys.path:
 METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 1 B200"
 
 # DRAM bytes (read + write) of one attention launch from an ncu capture (summaries under
-# profiles/), valid only for the kernel source they were captured on (md5 of
-# csrc/dp_attn_tc.cu); any other source reports null.
-TRAFFIC_SOURCE_MD5 = "4640b0b89f56c60bf7430dd4a1674f0a"
-TRAFFIC_BYTES = {"cogvideo_bf16": 232.817152e6 + 53.842432e6, "wan_bf16": 603.7056e6 + 141.67936e6}
+# profiles/), valid only for the kernel source they were captured on (md5 over
+# csrc/dp_attn_tc.cu and csrc/dp_device.cuh); any other source reports null.
+TRAFFIC_SOURCE_MD5 = "344a22bad7f73ba52e39afa38107bd22"
+TRAFFIC_BYTES = {"cogvideo_bf16": 232.528896e6 + 51.86304e6, "wan_bf16": 629.888768e6 + 143.290624e6}
 L2_BYTES = 126 * 1024 * 1024
 
 
 def attention_traffic(config_name: str):
     import hashlib
-    path = os.path.join(ROOT, "long_video_diffusion_b200", "csrc", "dp_attn_tc.cu")
-    try:
-        with open(path, "rb") as f:
-            md5 = hashlib.md5(f.read()).hexdigest()
-    except OSError:
-        return None
-    return TRAFFIC_BYTES.get(config_name) if md5 == TRAFFIC_SOURCE_MD5 else None
+    h = hashlib.md5()
+    for name in ("dp_attn_tc.cu", "dp_device.cuh"):
+        try:
+            with open(os.path.join(ROOT, "long_video_diffusion_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    return TRAFFIC_BYTES.get(config_name) if h.hexdigest() == TRAFFIC_SOURCE_MD5 else None
 
 
 def load_peaks():

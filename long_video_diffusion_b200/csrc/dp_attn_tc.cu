@@ -52,14 +52,9 @@ namespace dp {
 
 namespace {
 
-constexpr int BM = 128;       // query rows per tile
-constexpr int NQ = 2;         // query tiles per CTA
-constexpr int kThreads = 384; // 12 warps
-constexpr int kLaunchRegs = 168;  // 65536 / 384 rounded down to the allocation granule
-constexpr int kLowRegs = 72;
-constexpr int kHighRegs = 216;
-static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
+constexpr int BM = 128;          // query rows per tile
 constexpr int kTmemCols = 512;
+constexpr int kRegFile = 65536;  // 32-bit registers per SM
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
 // exp2 on the FMA pipe for part of the softmax (the MUFU unit retires 16 exp2 per clock per
@@ -83,39 +78,59 @@ struct PolyPairs {
 
 template <int HD>
 struct Layout {
-  // Keys per tile: 128 at head_dim 64; 64 at head_dim 128, so that P gets tensor-memory
-  // columns of its own there too (see below).  A 128x64x16 product costs about 3/4 of a
-  // 128x128x16 one on the tensor pipe, a smaller price than running each query tile's
-  // S -> softmax -> PV -> S chain strictly in series.
+  // Query tiles per CTA (one softmax warpgroup each) and keys per tile.  Tensor memory holds
+  // S_g (BN fp32 columns), P_g (BN/2 columns of 16-bit pairs) and O_g (HD columns) for each
+  // query tile: 128-key tiles at head_dim 64 (448 columns), 64-key tiles at head_dim 128
+  // (448 columns; 128-key tiles would leave no room for P, and each query tile would then
+  // run S -> softmax -> PV -> S strictly in series).  P therefore always has columns of its
+  // own, so the next S product runs while the softmax still works on the current tile.  A
+  // 128x64x16 product costs about 3/4 of a 128x128x16 one on the tensor pipe.  (Three query
+  // tiles of 64 keys also fit at head_dim 64; measured, they ran no faster per query tile
+  // and lost more to the last wave of CTAs.)
+  static constexpr int NQ = 2;
   static constexpr int BN = HD == 64 ? 128 : 64;
+  // warps: 4 per query tile (softmax), then the TMA producer, then three MMA issuers (the
+  // first also owns the tensor memory)
+  static constexpr int W_PROD = 4 * NQ;
+  static constexpr int W_ISS = W_PROD + 1;
+  static constexpr int kIssuers = 3;
+  static constexpr int kThreads = 32 * (W_PROD + 4);
+  static constexpr int kLaunchRegs = (kRegFile / kThreads) & ~7;  // the allocation granule is 8
+  // setmaxnreg: the producer/issuer warpgroup gives registers back, the softmax warpgroups
+  // take them (a softmax thread holds its row of S and P)
+  static constexpr int kLowRegs = 72;
+  static constexpr int kHighRegs = 216;
+  static_assert(NQ * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
   static constexpr int KCH = HD / 64;                    // 128-byte column chunks
   static constexpr int STAGES = 4;
   static constexpr int Q_CHUNK = BM * 128;               // one 64-column chunk of a Q tile
   static constexpr int KV_CHUNK = BN * 128;              // one 64-column chunk of a K or V tile
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
-  // Tensor memory: S_g (BN fp32 columns each), P_g (BN/2 columns of 16-bit pairs), O_g (HD
-  // columns).  When all of it fits, P has its own columns and the next S product can run
-  // while the softmax still works on the current tile; otherwise P is written over S_g.
-  // The wider of the S and O regions comes first, so every region starts at a multiple of
-  // its own width.
+  // When all of it fits, P has its own tensor-memory columns; otherwise P is written over
+  // S_g.  The wider of the S and O regions comes first, so every region starts at a
+  // multiple of its own width.
   static constexpr bool SEP_P = NQ * BN + NQ * (BN / 2) + NQ * HD <= kTmemCols;
-  static constexpr bool O_FIRST = HD > BN;
+  static constexpr bool O_FIRST = HD >= BN;
   static constexpr int COL_S = O_FIRST ? NQ * HD : 0;
   static constexpr int COL_P = SEP_P ? COL_S + NQ * BN : COL_S;
   static constexpr int P_STRIDE = SEP_P ? BN / 2 : BN;
   static constexpr int COL_O = O_FIRST ? 0 : (SEP_P ? COL_P + NQ * (BN / 2) : NQ * BN);
   static_assert(BN % 32 == 0 && (BN / 16 == 4 || BN / 16 == 8), "key tile width");
-  // Issue split (see the MMA issuers): one warp per query tile issues S when S has more
-  // products per key tile than PV (HD / 16 against BN / 16), else one warp per query tile
-  // issues PV.
-  static constexpr bool S_PER_G = HD > BN;
+  // Issue split (see the MMA issuers), so that each issuing warp issues the same number of
+  // products per key tile: one warp per query tile for whichever product has more
+  // instructions (HD / 16 for S against BN / 16 for PV), one warp for the other product of
+  // both tiles.
+  enum Split { kSPerTile, kPVPerTile };
+  static constexpr Split SPLIT = HD > BN ? kSPerTile : kPVPerTile;
+  static_assert(NQ == 2, "the issue split assumes two query tiles (three issuing warps)");
+  static constexpr int KV_EMPTY_ARRIVALS = SPLIT == kSPerTile ? 1 : NQ;  // PV-issuing warps
   static_assert((O_FIRST ? COL_P + NQ * P_STRIDE : COL_O + NQ * HD) <= kTmemCols, "tensor memory budget");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  // k_full[S], v_full[S], kv_empty[S], q_full[2], s_full[2], s_free[2], p_full[2], o_done[2], fin
+  // k_full[S], v_full[S], kv_empty[S], q_full[NQ], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ], fin
   static constexpr int N_BAR = 3 * STAGES + 5 * NQ + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -153,12 +168,13 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 template <int HD, bool F16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
     window_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                           const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
                           const Params p) {
   using L = Layout<HD>;
   constexpr int BN = L::BN;
+  constexpr int NQ = L::NQ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -185,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(v_full(s), 1);
-      mbar_init(kv_empty(s), L::S_PER_G ? 1 : NQ);  // one arrival from each PV issuing warp
+      mbar_init(kv_empty(s), L::KV_EMPTY_ARRIVALS);  // one arrival from each PV-issuing warp
     }
     for (int g = 0; g < NQ; ++g) {
       mbar_init(q_full(g), 128);
@@ -194,15 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full(g), 128);
       mbar_init(o_done(g), 1);
     }
-    mbar_init(fin, 1 + NQ);     // one arrival from each MMA issuer
+    mbar_init(fin, L::kIssuers);  // one arrival from each MMA issuer
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == L::W_ISS) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == L::W_PROD && lane == 0) {
     tma_prefetch_desc(&tm_kc);
     tma_prefetch_desc(&tm_vc);
     tma_prefetch_desc(&tm_kw);
@@ -213,9 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 8) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-  if (warp == 8) {
+  if (warp >= L::W_PROD) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::kLowRegs));
+  if (warp == L::W_PROD) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
@@ -300,9 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ts(d, pa + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idPV, (t > 0 || kk > 0) ? 1u : 0u);
       mma_commit(o_done(g));
     };
-    if constexpr (L::S_PER_G) {
-      if (warp == 9 || warp == 10) {
-        const int g = warp - 9;
+    const int iw = warp - L::W_ISS;  // issuing warp 0..2
+    if constexpr (L::SPLIT == L::kSPerTile) {
+      if (iw < NQ) {
+        const int g = iw;
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int st = t % L::STAGES;
           const uint32_t kpar = (t / L::STAGES) & 1;
@@ -315,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           mma_s(st, g);
         }
-      } else if (warp == 11) {
+      } else {
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int st = t % L::STAGES;
 #pragma unroll 1
@@ -329,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      if (warp == 9) {
+      if (iw == 0) {
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int st = t % L::STAGES;
 #pragma unroll 1
@@ -346,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_s(st, g);
           }
         }
-      } else if (warp == 10 || warp == 11) {
-        const int g = warp - 10;
+      } else {
+        const int g = iw - 1;
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int st = t % L::STAGES;
           ok = wait(p_full(g), t & 1, DEV_ERR_TIMEOUT_P) && wait(v_full(st), (t / L::STAGES) & 1, DEV_ERR_TIMEOUT_KV);
@@ -357,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (warp >= 9) {
+    if (warp >= L::W_ISS) {
       // every product this warp issued completes before TMEM is released
       mma_commit(fin);
       drain_wait(fin, 0, p.status);
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(L::kHighRegs));
     // ------------------------------------------------------------ softmax warpgroups
     const int g = warp >> 2;                       // query tile of this warpgroup
     const int t = threadIdx.x & 127;               // row within the tile
@@ -609,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == L::W_ISS) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -650,7 +667,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   p.n_win = a.n_win;
   p.cache_len = a.cache_len;
   p.hidden = a.hidden;
-  p.n_qpairs = static_cast<int32_t>((a.n_win + NQ * BM - 1) / (NQ * BM));
+  p.n_qpairs = static_cast<int32_t>((a.n_win + L::NQ * BM - 1) / (L::NQ * BM));
   p.n_ct = static_cast<int32_t>((a.cache_len + BN - 1) / BN);
   p.n_wt = static_cast<int32_t>((a.n_win + BN - 1) / BN);
   p.scale_log2 = a.softmax_scale * 1.4426950408889634f;
@@ -670,11 +687,11 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, window_attn_tc_kernel<HD, F16>);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+    if (fa.numRegs < L::kLaunchRegs) return cudaErrorInvalidConfiguration;
     attr_set[dev] = true;
   }
   const int64_t grid = static_cast<int64_t>(p.n_qpairs) * a.n_heads;
-  window_attn_tc_kernel<HD, F16><<<static_cast<unsigned>(grid), kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
+  window_attn_tc_kernel<HD, F16><<<static_cast<unsigned>(grid), L::kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
   return cudaGetLastError();
 }
 
