@@ -33,8 +33,8 @@ METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 
 # DRAM bytes (read + write) of one attention launch from an ncu capture (summaries under
 # profiles/), valid only for the kernel source they were captured on (md5 over
 # csrc/dp_attn_tc.cu and csrc/dp_device.cuh); any other source reports null.
-TRAFFIC_SOURCE_MD5 = "344a22bad7f73ba52e39afa38107bd22"
-TRAFFIC_BYTES = {"cogvideo_bf16": 232.528896e6 + 51.86304e6, "wan_bf16": 629.888768e6 + 143.290624e6}
+TRAFFIC_SOURCE_MD5 = "021dac6c4a1364996dd7c7e37e5b6f2e"
+TRAFFIC_BYTES = {"cogvideo_bf16": 232.533504e6 + 50.983424e6, "wan_bf16": 630.609152e6 + 142.060032e6}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -64,6 +64,9 @@ def load_peaks():
 
 def workload(name: str):
     from workloads import step_config
+    if name == "long_run":
+        # the oracle arms time a steady-state step of the run (same shapes as its 8-block window)
+        return step_config("longrun_steady_bf16")
     if name.startswith("sweep_"):
         parts = name.split("_")
         return step_config("sweep", int(parts[1]), ragged=len(parts) > 2 and parts[2] == "ragged")
@@ -225,6 +228,149 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
                      h2d=(hq.numel() + hk.numel() + hv.numel() + hnoise.numel()) * eb, d2h=hout.numel() * eb)
 
 
+def long_run_arm(args, rank: int, world: int, local_rank: int):
+    """The whole long-video queue run (257 latent frames, 8-block window, 50 staggered
+    timesteps per block): every schedule step is one window step of the library, with the
+    window growing from 1 to 8 blocks, the head block exiting into the cache and fresh noise
+    blocks pushed.  W warm-up steps run on a separate queue; then the first K schedule steps
+    (all 850 by default) of a fresh run are timed."""
+    import torch
+    import torch.distributed as dist
+
+    import long_video_diffusion_b200 as dp
+    from workloads import make_run_noise, make_run_table, run_config
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    rc = run_config()
+    H, hd, D, W, T = rc.n_heads, rc.head_dim, rc.hidden, rc.window_blocks, rc.n_timesteps
+    noise_cpu = make_run_noise(rc)
+    table = make_run_table(rc).to(dev)
+    noise = [b.to(dev) for b in noise_cpu]
+    tau = [int(round(999.0 * (T - 1 - i) / (T - 1))) for i in range(T)]
+    n_max = W * rc.slot_rows
+    kv = torch.empty(2 * n_max * D, dtype=torch.float16, device=dev)
+    out = torch.empty(n_max, D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fresh():
+        return dp.KVCache(rc.slot_rows, D, torch.float16, device=dev), dp.Queue(W, rc.slot_rows, D, device=dev)
+
+    cache, queue = fresh()
+    dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, max_steps=args.warmup)
+    torch.cuda.synchronize()
+    dp.device_status()
+
+    # per-step attention work: 4 n (L_c + n) hd H with L_c the cache length before the step
+    steps_n, steps_lc = [], []
+    cache, queue = fresh()
+    state = {"lc": 0}
+
+    launches = [0]
+
+    def on_step(step, n, popped, pushed):
+        steps_n.append(n)
+        steps_lc.append(state["lc"])
+        state["lc"] = cache.length
+        launches[0] += 2 + (1 if (popped or pushed is not None) else 0)   # modulate, attention (+ copy)
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(_smi_index(local_rank)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    dp.profile_begin(args.steps)
+    t0.record(stream)
+    n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    dp.device_status()
+    ms = t0.elapsed_time(t1)
+
+    # e2e: the same run through the public API with every pushed noise block copied from
+    # pinned host memory right before its push and every step's output read back to the host
+    class _HostBlocks:
+        def __init__(self, blocks):
+            self.host = [b.pin_memory() for b in blocks]
+            self.dev = torch.empty(rc.slot_rows, D, dtype=torch.bfloat16, device=dev)
+            self.h2d = 0
+
+        def __len__(self):
+            return len(self.host)
+
+        def __getitem__(self, i):
+            h = self.host[i]
+            self.dev[:h.shape[0]].copy_(h, non_blocking=True)
+            self.h2d += h.numel() * 2
+            return self.dev[:h.shape[0]]
+
+    hb = _HostBlocks(noise_cpu)
+    hout = torch.empty(n_max, D, dtype=torch.bfloat16).pin_memory()
+    d2h = [0]
+
+    def on_step_e2e(step, n, popped, pushed):
+        hout[:n].copy_(out[:n], non_blocking=True)
+        d2h[0] += n * D * 2
+
+    cache, queue = fresh()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    dp.device_status()
+    tokens = sum(steps_n)
+    flop = sum(4 * n * (lc + n) * hd * H for n, lc in zip(steps_n, steps_lc))
+    ms, e2e_ms, attn_ms = max_over_ranks([ms, e2e_ms, attn_ms], dev)
+    return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
+                e2e_ms=e2e_ms, e2e_steps=n_e2e, h2d=hb.h2d / max(n_e2e, 1), d2h=d2h[0] / max(n_e2e, 1),
+                clocks=clocks, rc=rc, launches=launches[0])
+
+
+def long_run_line(args, world, r):
+    peaks = load_peaks()
+    rc = r["rc"]
+    achieved = r["flop"] / (r["attn_ms"] / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    steady_flop = 4 * 21600 * (21600 + 2700) * rc.head_dim * rc.n_heads
+    return {
+        "metric": METRIC, "value": world * r["tokens"] / (r["ms"] / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": r["steps"], "warmup": args.warmup, "ms_per_step": r["ms"] / r["steps"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"long_run: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
+                                f"{rc.frames_per_block}-frame blocks, window of {rc.window_blocks} blocks, "
+                                f"{rc.n_timesteps} staggered timesteps per block, {rc.n_heads}x{rc.head_dim} heads, "
+                                f"bf16; first {r['steps']} schedule steps"),
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "steady-state window q = k = v 66 MiB plus k', v', cache and out: 265 MiB per step > 126 MiB"},
+        "window_tokens": r["tokens"],
+        "attn_tflops": achieved,
+        "stage_ms": {"modulate": r["mod_ms"] / r["steps"], "attention": r["attn_ms"] / r["steps"],
+                     "advance": r["adv_ms"] / r["steps"]},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "traffic_unit": "bytes per launch (not captured for the run: window sizes vary per step)",
+                     "kernel": "window_attn_tc_kernel",
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "algorithmic_flop_per_run": r["flop"], "steady_state_flop_per_launch": steady_flop},
+        "clocks": r["clocks"],
+        "e2e": {"value": world * r["tokens"] / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": None,
+    }
+
+
 def stage_hbm(cfg, r, peaks):
     """Achieved HBM bandwidth of the two copy-like stages (algorithmic bytes / event time):
     modulation reads k, v and writes k', v' (4 N_w D e bytes); the advance copies the head
@@ -383,10 +529,23 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    try:
-        cfg, r = gpu_arm(args, rank, world, local_rank)
-    finally:
-        pass
+    if args.config == "long_run":
+        if args.steps == 300 and "--steps" not in sys.argv:
+            args.steps = 850                 # the whole run
+        r = long_run_arm(args, rank, world, local_rank)
+        if rank == 0:
+            line = long_run_line(args, world, r)
+            line["gpu_launches"] = r["launches"] if "launches" in r else None
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(workload("long_run"))
+                line["cpu_baseline"]["sample"] = "steady-state step of the run: " + line["cpu_baseline"]["sample"]
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    cfg, r = gpu_arm(args, rank, world, local_rank)
     if rank == 0:
         peaks = load_peaks()
         flop = cfg.attn_flop()

@@ -365,18 +365,19 @@ def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
 
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
              queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
-             on_step=None, stream=None) -> int:
+             on_step=None, stream=None, max_steps: Optional[int] = None) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
     noise_blocks: device tensors in entry order.  on_step(step, n_win, popped, pushed) is
-    called after each step is enqueued.  Returns the number of steps."""
+    called after each step is enqueued.  max_steps stops the run early (the queue and cache
+    are then left mid-run).  Returns the number of steps."""
     T = len(tau)
     n_blocks = len(noise_blocks)
     queue_push(queue, noise_blocks[0], stream=stream)
     nxt = 1
     step = 0
-    while queue.count > 0:
+    while queue.count > 0 and (max_steps is None or step < max_steps):
         blk, win, n = queue_blocks(queue, table, tau)
         pop = queue.evals()[0] + 1 == T
         push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1

@@ -32,6 +32,10 @@ def test_config_timesteps_and_sizes():
     assert c2.timesteps == [0, 143, 285, 428, 571, 714, 856, 999]
     assert c2.n_win == 49920 and c2.cache_len == 6240 and c2.hidden == 1536
     assert c1.attn_flop() == 4 * 10800 * 13500 * 64 * 48
+    c3 = step_config("longrun_steady_bf16")
+    rc = run_config()
+    assert c3.block_rows == [rc.slot_rows] * rc.window_blocks and c3.cache_len == rc.slot_rows
+    assert (c3.n_heads, c3.head_dim) == (rc.n_heads, rc.head_dim) and c3.n_win == 21600
     sw = sweep_configs()
     assert [c.n_win for c in sw[:2]] == [4096, 3840]
     assert sw[-1].cache_len == 131072 // 4 and sw[-1].block_rows == [32768, 32768, 32768, 24576]

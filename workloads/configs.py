@@ -11,6 +11,8 @@ block that left) plus the five workload definitions this library is measured on:
                     cache, 12x128 heads, bf16.
 * ``long_run``      257 latent frames x 1350 tokens in 2-frame blocks, window of 8
                     blocks, 50 staggered timesteps per block, 24x64 heads, bf16.
+* ``longrun_steady_bf16``  one window step of the long run's steady state: 8 blocks x
+                    2700 tokens, 2700-token cache, 24x64 heads, N(0,1) inputs.
 * ``sweep``         window of 4 blocks, 4096..131072 tokens, cache = window/4,
                     16x128 heads, bf16, with a ragged last block variant.
 
@@ -24,7 +26,7 @@ from typing import List, Optional
 
 SEED_BASE = 20250527
 
-CONFIG_NAMES = ["tiny_f32", "cogvideo_bf16", "wan_bf16", "long_run", "sweep"]
+CONFIG_NAMES = ["tiny_f32", "cogvideo_bf16", "wan_bf16", "long_run", "longrun_steady_bf16", "sweep"]
 
 
 @dataclass
@@ -124,6 +126,10 @@ def step_config(name: str, n: Optional[int] = None, ragged: bool = False) -> Ste
         return StepConfig(name, "bf16", 12, 128, [6240] * 8, 6240, 6240, _even_timesteps(8),
                           1.0, SEED_BASE + 2, push_rows=6240,
                           note="Wan-like 832x480: 1560 tokens per latent frame")
+    if name == "longrun_steady_bf16":
+        return StepConfig(name, "bf16", 24, 64, [2700] * 8, 2700, 2700, _even_timesteps(8),
+                          1.0, SEED_BASE + 6, push_rows=2700,
+                          note="steady state of the long run: 8 blocks of 2 latent frames x 1350 tokens")
     if name == "sweep":
         if n is None:
             raise ValueError("sweep needs n (window tokens)")
