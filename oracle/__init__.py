@@ -28,11 +28,20 @@ Parity status of each function (how it is pinned, in tests/test_oracle_pins.py):
   long_run_schedule pinned: every block evaluated exactly T times in timestep order,
                     at most W live, exit of block b coincides with entry of b + W,
                     noise level monotone along the queue
+  layer_norm        pinned: hand-computed row; zero mean and variance var/(var + eps);
+                    a constant row maps to zero; brute-force loops
+  ln_modulate       pinned: zero shift/scale -> layer_norm; scale = -1 -> shift_b
+  linear            pinned: brute-force loops; identity weights -> a + bias
+  round_to          pinned: hand-computed bf16/f16 bit patterns, f16 saturation
+  sublayer_step     pinned: identity projections reduce it to x + gated window_attention
+                    of the normed window; brute-force loops end to end on tiny inputs
 """
 from .dualparal import (as_f64, row_blocks, lookup, modulate, modulate_rounded,
                         window_attention, window_step, KVCacheRing, FifoQueue,
                         entry_step, long_run_schedule, timestep_schedule, LongRun)
+from .sublayer import round_to, layer_norm, ln_modulate, linear, sublayer_step
 
 __all__ = ["as_f64", "row_blocks", "lookup", "modulate", "modulate_rounded",
            "window_attention", "window_step", "KVCacheRing", "FifoQueue", "entry_step",
-           "long_run_schedule", "timestep_schedule", "LongRun"]
+           "long_run_schedule", "timestep_schedule", "LongRun", "round_to", "layer_norm",
+           "ln_modulate", "linear", "sublayer_step"]

@@ -209,7 +209,7 @@ def test_window_step_tiny_f32_two_steps(dp):
     assert errors(out2.cpu().double().numpy(), want)[0] > 1e-3   # the cache did change the result
 
 
-@pytest.mark.parametrize("name", ["cogvideo_bf16", "wan_bf16"])
+@pytest.mark.parametrize("name", ["cogvideo_bf16", "wan_bf16", "longrun_steady_bf16", "wan_paper_bf16"])
 def test_window_step_full_size_sampled(dp, name):
     """Full-size bf16 step in the launch configuration the benchmark times; the oracle
     computes sampled rows (block boundaries, first/last, ragged tail, random)."""

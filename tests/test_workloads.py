@@ -36,6 +36,8 @@ def test_config_timesteps_and_sizes():
     rc = run_config()
     assert c3.block_rows == [rc.slot_rows] * rc.window_blocks and c3.cache_len == rc.slot_rows
     assert (c3.n_heads, c3.head_dim) == (rc.n_heads, rc.head_dim) and c3.n_win == 21600
+    c4 = step_config("wan_paper_bf16")
+    assert c4.block_rows == [8 * 1560] * 4 and c4.cache_len == 8 * 1560 and c4.hidden == 1536
     sw = sweep_configs()
     assert [c.n_win for c in sw[:2]] == [4096, 3840]
     assert sw[-1].cache_len == 131072 // 4 and sw[-1].block_rows == [32768, 32768, 32768, 24576]

@@ -7,8 +7,9 @@ can consume the same inputs without sharing any code that computes results.
 """
 from .configs import (StepConfig, RunConfig, step_config, run_config, sweep_configs,
                       CONFIG_NAMES)
-from .gen import make_step_inputs, make_run_noise, make_run_table, to_dtype, as_features
+from .gen import (make_step_inputs, make_run_noise, make_run_table, to_dtype, as_features,
+                  make_sublayer_weights)
 
 __all__ = ["StepConfig", "RunConfig", "step_config", "run_config", "sweep_configs",
            "CONFIG_NAMES", "make_step_inputs", "make_run_noise", "make_run_table",
-           "to_dtype", "as_features"]
+           "to_dtype", "as_features", "make_sublayer_weights"]

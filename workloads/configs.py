@@ -13,6 +13,9 @@ block that left) plus the five workload definitions this library is measured on:
                     blocks, 50 staggered timesteps per block, 24x64 heads, bf16.
 * ``longrun_steady_bf16``  one window step of the long run's steady state: 8 blocks x
                     2700 tokens, 2700-token cache, 24x64 heads, N(0,1) inputs.
+* ``wan_paper_bf16`` the pages' own block size on the Wan-like latent: 4 blocks of 8 latent
+                    frames x 1560 tokens, a cache of 8 latent frames (one exited block),
+                    12x128 heads, bf16.
 * ``sweep``         window of 4 blocks, 4096..131072 tokens, cache = window/4,
                     16x128 heads, bf16, with a ragged last block variant.
 
@@ -26,7 +29,7 @@ from typing import List, Optional
 
 SEED_BASE = 20250527
 
-CONFIG_NAMES = ["tiny_f32", "cogvideo_bf16", "wan_bf16", "long_run", "longrun_steady_bf16", "sweep"]
+CONFIG_NAMES = ["tiny_f32", "cogvideo_bf16", "wan_bf16", "long_run", "longrun_steady_bf16", "wan_paper_bf16", "sweep"]
 
 
 @dataclass
@@ -130,6 +133,10 @@ def step_config(name: str, n: Optional[int] = None, ragged: bool = False) -> Ste
         return StepConfig(name, "bf16", 24, 64, [2700] * 8, 2700, 2700, _even_timesteps(8),
                           1.0, SEED_BASE + 6, push_rows=2700,
                           note="steady state of the long run: 8 blocks of 2 latent frames x 1350 tokens")
+    if name == "wan_paper_bf16":
+        return StepConfig(name, "bf16", 12, 128, [12480] * 4, 12480, 12480, _even_timesteps(4),
+                          1.0, SEED_BASE + 7, push_rows=12480,
+                          note="blocks of 8 latent frames (the pages' block boundaries and 8-frame context)")
     if name == "sweep":
         if n is None:
             raise ValueError("sweep needs n (window tokens)")

@@ -71,3 +71,17 @@ def make_run_noise(cfg: RunConfig, dtype: str = "bf16") -> List[torch.Tensor]:
     g = torch.Generator().manual_seed(cfg.seed)
     _randn(g, (cfg.table_rows, 3, cfg.hidden))  # advance past the table draw
     return [to_dtype(_randn(g, (rows, cfg.hidden)), dtype) for rows in cfg.block_rows]
+
+
+def make_sublayer_weights(hidden: int, seed: int) -> Dict[str, torch.Tensor]:
+    """Seeded stand-in weights of the DiT attention sublayer (trained weights are out of
+    reach): W_qkv [3 hidden][hidden] and W_o [hidden][hidden] (out-features x in-features)
+    drawn N(0, 1/hidden) so unit-variance inputs give unit-variance outputs, rounded once
+    to bf16; biases N(0, 0.02^2) in float32.  Draw order: W_qkv, b_qkv, W_o, b_o."""
+    g = torch.Generator().manual_seed(seed)
+    s = 1.0 / float(hidden) ** 0.5
+    w_qkv = _randn(g, (3 * hidden, hidden), s).to(torch.bfloat16).contiguous()
+    b_qkv = _randn(g, (3 * hidden,), 0.02).contiguous()
+    w_o = _randn(g, (hidden, hidden), s).to(torch.bfloat16).contiguous()
+    b_o = _randn(g, (hidden,), 0.02).contiguous()
+    return {"w_qkv": w_qkv, "b_qkv": b_qkv, "w_o": w_o, "b_o": b_o}
