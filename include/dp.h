@@ -15,6 +15,9 @@
  *       prologue and the gate (+ residual) into its epilogue   dp_window_attention
  *   A3  queue and cache advance               dp_kvcache_advance, dp_queue_push/pop
  *   A4  the whole step A1 -> A2 -> A3         dp_window_step
+ *   B   the DiT attention sublayer around A2 (pre-norm, q/k/v and output projections on
+ *       caller-supplied weights): dp_ln_modulate, dp_linear, dp_qkv_project,
+ *       dp_out_project, dp_sublayer_step
  *
  * Conventions (all entry points):
  *  - Token tensors are row-major [rows][hidden], hidden = n_heads * head_dim, channel
@@ -249,10 +252,71 @@ dp_status dp_window_step_noalloc(const void* q, const void* k, const void* v, in
                                  dp_queue* queue, const void* push_noise, int64_t push_rows,
                                  dp_dtype dt, void* stream);
 
+/* ---------------------------------------------------------------- B: DiT attention sublayer */
+
+/*
+ * The DiT layer around the window attention, with the adaLN conditioning of the pages'
+ * DiT (the review's Section 3.1: each block is denoised at its own timestep; Section 3.2:
+ * the self-attention K/V of the block that left are cached):
+ *   B1  h   = LN(x) * (1 + scale_b) + shift_b          dp_ln_modulate
+ *   B2  q, k, v = h W_qkv^T + b_qkv                     dp_qkv_project (dp_linear: plain)
+ *   A2  o   = attention over [cache ; window k, v]     dp_window_attention, no flags
+ *   B3  out = x + gate_b * (o W_o^T + b_o)              dp_out_project
+ *   B4  the whole sublayer step and its advance         dp_sublayer_step
+ * Weights are the caller's (trained weights are not part of this library): W_qkv DEVICE
+ * [3 * hidden][hidden] bf16 and W_o [hidden][hidden] bf16, out-features by in-features
+ * (row i of W holds output feature i's input weights), biases DEVICE float [3 * hidden] /
+ * [hidden] or NULL.  Products run on the tensor cores with fp32 accumulation.
+ */
+
+/* B1: h_i = (x_i - mean_i) / sqrt(var_i + eps) * (1 + scale_b) + shift_b, mean and (biased)
+ * variance over the row's hidden channels, computed in fp32 (two passes) and rounded once
+ * to bf16; b = block of row i.  x, h: DEVICE [n_rows][hidden] bf16, h may equal x.
+ * hidden = blk->hidden must be a multiple of 256 and at most 8192 (UNSUPPORTED
+ * otherwise); eps > 0. */
+dp_status dp_ln_modulate(const void* x, void* h, int64_t n_rows, const dp_blocks* blk, float eps,
+                         void* stream);
+
+/* y = a W^T + bias: a DEVICE [m][k] bf16, w DEVICE [n][k] bf16, bias DEVICE [n] float or
+ * NULL, y DEVICE [m][n] of y_dt (bf16, or f16 saturating at +-65504), rounded once from
+ * the fp32 sum (round to nearest even).  n a multiple of 128 and k of 8 (UNSUPPORTED
+ * otherwise).  y overlaps no input. */
+dp_status dp_linear(const void* a, const void* w, const float* bias, int64_t m, int32_t n,
+                    int32_t k, void* y, dp_dtype y_dt, void* stream);
+
+/* B2: [q | k | v] = h W_qkv^T + b_qkv, split by output column: q (columns [0, hidden))
+ * DEVICE [n_rows][hidden] bf16 (the attention's raw query), k and v (columns [hidden,
+ * 2 hidden) and [2 hidden, 3 hidden)) DEVICE [n_rows][hidden] f16 features (saturating).
+ * hidden a multiple of 128. */
+dp_status dp_qkv_project(const void* h, const void* w_qkv, const float* b_qkv, int64_t n_rows,
+                         int32_t hidden, void* q, void* k, void* v, void* stream);
+
+/* B3: out_i = residual_i + gate_b * (o_i W_o^T + b_o), b = block of row i, gate from
+ * blk->mod[b] (after shift and scale), all in fp32, rounded once to bf16.  o, residual,
+ * out: DEVICE [n_rows][hidden] bf16, hidden = blk->hidden a multiple of 128; out overlaps
+ * no input. */
+dp_status dp_out_project(const void* o, const void* w_o, const float* b_o, int64_t n_rows,
+                         const dp_blocks* blk, const void* residual, void* out, void* stream);
+
+/* B4: one sublayer step on the window x (DEVICE [n_win][hidden] bf16, e.g. the queue's
+ * live window): B1, B2, the attention over [cache ; k, v] (softmax scale 1/sqrt(head_dim),
+ * no modulation or gate inside it), B3 into out, then the advance of dp_window_step: every
+ * live block's evals += 1; with DP_STEP_POP the head block's k and v rows (the projected
+ * features of its last evaluation) become the cache and the queue pops; push_noise is
+ * pushed at the tail.  work: DEVICE scratch of 4 * n_win * hidden 16-bit elements (h and
+ * then the attention output, q, k, v); the cache holds f16 features; head_dim 64 or 128;
+ * hidden a multiple of 256.  out overlaps neither x nor work.  All checks happen before
+ * anything is enqueued. */
+dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, const void* w_qkv,
+                           const float* b_qkv, const void* w_o, const float* b_o, float eps,
+                           dp_kvcache* cache, void* work, void* out, int32_t n_heads,
+                           int32_t head_dim, uint32_t flags, dp_queue* queue,
+                           const void* push_noise, int64_t push_rows, void* stream);
+
 /* ---------------------------------------------------------------- profiling */
 
-/* Stage timing of dp_window_step.  After dp_profile_begin(max_steps), the next max_steps
- * dp_window_step calls on this thread record CUDA events (created and owned by the
+/* Stage timing of dp_window_step and dp_sublayer_step.  After dp_profile_begin(max_steps),
+ * the next max_steps such calls on this thread record CUDA events (created and owned by the
  * library; no device memory) on their stream at the boundaries of the modulation prepass,
  * the attention and the advance.  dp_profile_end synchronizes on the last recorded event,
  * returns the summed times in milliseconds (any output pointer may be NULL) and the number
@@ -261,6 +325,12 @@ dp_status dp_window_step_noalloc(const void* q, const void* k, const void* v, in
 dp_status dp_profile_begin(int32_t max_steps);
 dp_status dp_profile_end(float* ms_modulate, float* ms_attention, float* ms_advance,
                          int32_t* steps);
+/* The same for any recorded step kind: ms[i] (i < max_stages) receives stage i's summed
+ * time — for dp_window_step 0 modulation, 1 attention, 2 advance; for dp_sublayer_step
+ * 0 pre-norm and modulation, 1 q/k/v projection, 2 attention, 3 out projection,
+ * 4 advance — *n_stages the most stages any recorded step had. */
+dp_status dp_profile_end_stages(float* ms, int32_t max_stages, int32_t* n_stages,
+                                int32_t* steps);
 
 /* ---------------------------------------------------------------- status */
 

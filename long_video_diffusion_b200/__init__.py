@@ -80,8 +80,15 @@ _SIGS = {
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
     "dp_window_step_noalloc": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P,
                                _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
+    "dp_ln_modulate": [_P, _P, _I64, ctypes.POINTER(DpBlocks), _F, _P],
+    "dp_linear": [_P, _P, _P, _I64, _I32, _I32, _P, _I32, _P],
+    "dp_qkv_project": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P],
+    "dp_out_project": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), _P, _P, _P],
+    "dp_sublayer_step": [_P, _I64, ctypes.POINTER(DpBlocks), _P, _P, _P, _P, _F, ctypes.POINTER(DpKvcache), _P, _P,
+                         _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _P],
     "dp_profile_begin": [_I32],
     "dp_profile_end": [ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_I32)],
+    "dp_profile_end_stages": [ctypes.POINTER(_F), _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I32)],
     "dp_set_device": [_I32],
     "dp_device_status": [_P],
     "dp_status_string": [_I32],
@@ -304,6 +311,68 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
                                int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
 
 
+# ------------------------------------------------------------------------- B: DiT attention sublayer
+
+LN_EPS = 1e-6
+
+
+def ln_modulate(x, h, blocks: DpBlocks, eps: float = LN_EPS, stream=None) -> None:
+    """h = LN(x) * (1 + scale_b) + shift_b (dp_ln_modulate); x, h bf16 [rows][hidden]."""
+    _check(_lib.dp_ln_modulate(_ptr(x), _ptr(h), x.shape[0], ctypes.byref(blocks), float(eps), _stream(x, stream)),
+           "dp_ln_modulate")
+
+
+def linear(a, w, bias, y, stream=None) -> None:
+    """y = a W^T + bias on the tensor cores (dp_linear); a [m][k] and w [n][k] bf16, bias
+    float [n] or None, y bf16 or f16 [m][n]."""
+    _check(_lib.dp_linear(_ptr(a), _ptr(w), _ptr(bias), a.shape[0], w.shape[0], a.shape[1], _ptr(y), _dtype(y),
+                          _stream(a, stream)), "dp_linear")
+
+
+def qkv_project(h, w_qkv, b_qkv, q, k, v, stream=None) -> None:
+    """[q | k | v] = h W_qkv^T + b_qkv (dp_qkv_project): q bf16, k and v f16."""
+    _check(_lib.dp_qkv_project(_ptr(h), _ptr(w_qkv), _ptr(b_qkv), h.shape[0], h.shape[1], _ptr(q), _ptr(k), _ptr(v),
+                               _stream(h, stream)), "dp_qkv_project")
+
+
+def out_project(o, w_o, b_o, blocks: DpBlocks, residual, out, stream=None) -> None:
+    """out = residual + gate_b * (o W_o^T + b_o) (dp_out_project), bf16."""
+    _check(_lib.dp_out_project(_ptr(o), _ptr(w_o), _ptr(b_o), o.shape[0], ctypes.byref(blocks), _ptr(residual),
+                               _ptr(out), _stream(o, stream)), "dp_out_project")
+
+
+def sublayer_work(n_win: int, hidden: int, device=None) -> torch.Tensor:
+    """Scratch for sublayer_step: h / attention output, q, k, v (16-bit, n_win x hidden each)."""
+    return torch.empty(4 * n_win * hidden, dtype=torch.bfloat16, device=device or "cuda")
+
+
+def sublayer_step(x, blocks: DpBlocks, w_qkv, b_qkv, w_o, b_o, cache: KVCache, work, out, n_heads: int,
+                  head_dim: int, eps: float = LN_EPS, pop: bool = False, queue: Optional[Queue] = None,
+                  push_noise=None, push_rows=None, stream=None, n_win: Optional[int] = None) -> None:
+    """One DiT attention-sublayer step (dp_sublayer_step).  x is a tensor or a raw device
+    address (n_win then required), e.g. the queue's live window; work from sublayer_work.
+    After the call, work's planes 2 and 3 hold the window's projected k and v (f16)."""
+    if isinstance(x, torch.Tensor):
+        ref, n, xp = x, x.shape[0], _ptr(x)
+    else:
+        ref, n, xp = out, int(n_win), ctypes.c_void_p(x)
+    rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
+    _check(_lib.dp_sublayer_step(xp, n, ctypes.byref(blocks), _ptr(w_qkv), _ptr(b_qkv), _ptr(w_o), _ptr(b_o),
+                                 float(eps), ctypes.byref(cache.desc), _ptr(work), _ptr(out), n_heads, head_dim,
+                                 STEP_POP if pop else 0, ctypes.byref(queue.desc) if queue is not None else None,
+                                 _ptr(push_noise), int(rows), _stream(ref, stream)), "dp_sublayer_step")
+
+
+def sublayer_planes(work, n_win: int, hidden: int):
+    """Views of the sublayer scratch: (o, q, k, v), each [n_win][hidden]."""
+    plane = n_win * hidden
+    o = work[:plane].view(n_win, hidden)
+    q = work[plane:2 * plane].view(n_win, hidden)
+    k = work[2 * plane:3 * plane].view(torch.float16).view(n_win, hidden)
+    v = work[3 * plane:4 * plane].view(torch.float16).view(n_win, hidden)
+    return o, q, k, v
+
+
 def profile_begin(max_steps: int) -> None:
     """Time the stages of the next max_steps window_step calls on this thread."""
     _check(_lib.dp_profile_begin(int(max_steps)), "dp_profile_begin")
@@ -316,6 +385,16 @@ def profile_end():
     _check(_lib.dp_profile_end(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(n)),
            "dp_profile_end")
     return a.value, b.value, c.value, n.value
+
+
+def profile_end_stages(max_stages: int = 5):
+    """([ms per stage], n_stages, steps) summed since profile_begin (dp_profile_end_stages):
+    window steps 0 modulation, 1 attention, 2 advance; sublayer steps 0 pre-norm, 1 q/k/v
+    projection, 2 attention, 3 out projection, 4 advance."""
+    ms = (_F * max_stages)()
+    ns, n = ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.dp_profile_end_stages(ms, max_stages, ctypes.byref(ns), ctypes.byref(n)), "dp_profile_end_stages")
+    return [ms[i] for i in range(max_stages)], ns.value, n.value
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

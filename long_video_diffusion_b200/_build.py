@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libdp_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
-SOURCES = ["dp_api.cu", "dp_attn_tc.cu", "dp_attn_f32.cu", "dp_modulate.cu", "dp_noalloc.cu"]
+SOURCES = ["dp_api.cu", "dp_attn_tc.cu", "dp_attn_f32.cu", "dp_gemm.cu", "dp_modulate.cu", "dp_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-shared",
          "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]

@@ -15,9 +15,12 @@
 namespace {
 
 thread_local char g_detail[512] = "";
-// Stage profiling of dp_window_step (per thread): 4 events per recorded step.
+// Stage profiling of dp_window_step and dp_sublayer_step (per thread): up to kProfEvents
+// events per recorded step (stage boundaries), nst[i] stages in step i.
+constexpr int kProfEvents = 6;
 struct Profile {
   std::vector<cudaEvent_t> ev;
+  std::vector<int> nst;
   int32_t max_steps = 0;
   int32_t count = 0;
   bool active = false;
@@ -26,7 +29,14 @@ thread_local Profile g_prof;
 
 cudaEvent_t prof_event(int stage) {
   if (!g_prof.active || g_prof.count >= g_prof.max_steps) return nullptr;
-  return g_prof.ev[4 * g_prof.count + stage];
+  return g_prof.ev[kProfEvents * g_prof.count + stage];
+}
+
+// A step that recorded its events counts once it has recorded the last one.
+void prof_step_done(cudaEvent_t last, int n_stages) {
+  if (!last) return;
+  g_prof.nst[g_prof.count] = n_stages;
+  g_prof.count += 1;
 }
 
 cudaError_t record(cudaEvent_t ev, cudaStream_t s) { return ev ? cudaEventRecord(ev, s) : cudaSuccess; }
@@ -211,7 +221,8 @@ const char* dp_last_error_detail(void) { return g_detail; }
 dp_status dp_profile_begin(int32_t max_steps) {
   if (max_steps < 1) return fail(DP_ERR_INVALID_ARG, "max_steps %d", max_steps);
   if (g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling already active");
-  g_prof.ev.assign(static_cast<size_t>(4) * max_steps, nullptr);
+  g_prof.ev.assign(static_cast<size_t>(kProfEvents) * max_steps, nullptr);
+  g_prof.nst.assign(static_cast<size_t>(max_steps), 0);
   for (auto& e : g_prof.ev) {
     cudaError_t r = cudaEventCreate(&e);
     if (r != cudaSuccess) {
@@ -227,27 +238,59 @@ dp_status dp_profile_begin(int32_t max_steps) {
   return DP_OK;
 }
 
-dp_status dp_profile_end(float* ms_modulate, float* ms_attention, float* ms_advance, int32_t* steps) {
+namespace {
+
+// Per-stage sums (ms) over the recorded steps, then the events are released.
+dp_status profile_collect(double (&sum)[kProfEvents - 1], int* n_stages) {
   if (!g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling not active");
-  double sum[3] = {0.0, 0.0, 0.0};
+  for (double& x : sum) x = 0.0;
+  *n_stages = 0;
   dp_status st = DP_OK;
   if (g_prof.count > 0) {
-    cudaError_t r = cudaEventSynchronize(g_prof.ev[4 * (g_prof.count - 1) + 3]);
-    for (int i = 0; r == cudaSuccess && i < g_prof.count; ++i)
-      for (int k = 0; r == cudaSuccess && k < 3; ++k) {
+    const int last = g_prof.count - 1;
+    cudaError_t r = cudaEventSynchronize(g_prof.ev[kProfEvents * last + g_prof.nst[last]]);
+    for (int i = 0; r == cudaSuccess && i < g_prof.count; ++i) {
+      *n_stages = g_prof.nst[i] > *n_stages ? g_prof.nst[i] : *n_stages;
+      for (int k = 0; r == cudaSuccess && k < g_prof.nst[i]; ++k) {
         float ms = 0.0f;
-        r = cudaEventElapsedTime(&ms, g_prof.ev[4 * i + k], g_prof.ev[4 * i + k + 1]);
+        r = cudaEventElapsedTime(&ms, g_prof.ev[kProfEvents * i + k], g_prof.ev[kProfEvents * i + k + 1]);
         sum[k] += ms;
       }
+    }
     if (r != cudaSuccess) st = cuda_fail(r, "event timing");
   }
   for (auto& e : g_prof.ev) cudaEventDestroy(e);
   g_prof.ev.clear();
+  g_prof.nst.clear();
   g_prof.active = false;
+  return st;
+}
+
+}  // namespace
+
+dp_status dp_profile_end(float* ms_modulate, float* ms_attention, float* ms_advance, int32_t* steps) {
+  if (!g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling not active");
+  double sum[kProfEvents - 1];
+  int n_stages = 0;
+  const int32_t count = g_prof.count;
+  dp_status st = profile_collect(sum, &n_stages);
   if (ms_modulate) *ms_modulate = static_cast<float>(sum[0]);
   if (ms_attention) *ms_attention = static_cast<float>(sum[1]);
   if (ms_advance) *ms_advance = static_cast<float>(sum[2]);
-  if (steps) *steps = g_prof.count;
+  if (steps) *steps = count;
+  return st;
+}
+
+dp_status dp_profile_end_stages(float* ms, int32_t max_stages, int32_t* n_stages, int32_t* steps) {
+  if (!g_prof.active) return fail(DP_ERR_INVALID_ARG, "profiling not active");
+  double sum[kProfEvents - 1];
+  int ns = 0;
+  const int32_t count = g_prof.count;
+  dp_status st = profile_collect(sum, &ns);
+  if (ms)
+    for (int k = 0; k < max_stages && k < kProfEvents - 1; ++k) ms[k] = static_cast<float>(sum[k]);
+  if (n_stages) *n_stages = ns;
+  if (steps) *steps = count;
   return st;
 }
 
@@ -530,7 +573,232 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   }
   e = record(ev3, s);
   if (e != cudaSuccess) return cuda_fail(e, "event record");
-  if (ev3) g_prof.count += 1;
+  prof_step_done(ev3, 3);
+  if (queue)
+    for (int i = 0; i < queue->count; ++i) queue->evals[i] += 1;
+  if (pop) {
+    cache->len[wslot] = n_exit;
+    cache->n_advances += 1;
+    if (queue) apply_pop(queue);
+  }
+  if (push_noise) apply_push(queue, push_rows);
+  return DP_OK;
+}
+
+
+// ------------------------------------------------------------------ B: DiT attention sublayer
+
+namespace {
+
+// GEMM operand checks shared by the linear entry points: a [m][k] bf16, w [n][k] bf16.
+dp_status check_linear(const void* a, const void* w, const float* bias, int64_t m, int64_t n, int64_t k) {
+  if (!a || !w) return fail(DP_ERR_INVALID_ARG, "a/w NULL");
+  if (!aligned16(a) || !aligned16(w) || (bias && !aligned16(bias)))
+    return fail(DP_ERR_INVALID_ARG, "a/w/bias not 16-byte aligned");
+  if (m <= 0 || m > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "m %lld", static_cast<long long>(m));
+  if (n <= 0 || n % 128 || n > INT32_MAX)
+    return fail(DP_ERR_UNSUPPORTED, "n %lld (a positive multiple of 128)", static_cast<long long>(n));
+  if (k <= 0 || k % 8 || k > INT32_MAX)
+    return fail(DP_ERR_UNSUPPORTED, "k %lld (a positive multiple of 8)", static_cast<long long>(k));
+  return DP_OK;
+}
+
+dp_status run_gemm(dp::GemmArgs& g, cudaStream_t s, const char* what) {
+  dp_status st = status_ptr(&g.status);
+  if (st != DP_OK) return st;
+  cudaError_t e = dp::launch_gemm(g, s);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return DP_OK;
+}
+
+dp::GemmArgs gemm_args(const void* a, const void* w, const float* bias, int64_t m, int32_t n, int32_t k, int epi) {
+  dp::GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.a = a;
+  g.w = w;
+  g.bias = bias;
+  g.m = m;
+  g.n = n;
+  g.k = k;
+  g.epi = epi;
+  return g;
+}
+
+dp_status check_ln(const void* x, const void* h, int64_t n_rows, const dp_blocks* blk, float eps) {
+  if (!x || !h || !aligned16(x) || !aligned16(h)) return fail(DP_ERR_INVALID_ARG, "x/h NULL or misaligned");
+  if (!blk) return fail(DP_ERR_INVALID_ARG, "block table is NULL");
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return fail(DP_ERR_INVALID_ARG, "eps must be positive");
+  if (n_rows <= 0 || n_rows > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_rows %lld", static_cast<long long>(n_rows));
+  if (blk->hidden % 256 || blk->hidden <= 0 || blk->hidden > 8192)
+    return fail(DP_ERR_UNSUPPORTED, "hidden %d (a multiple of 256, at most 8192)", blk->hidden);
+  return check_blocks(blk, n_rows, blk->hidden);
+}
+
+dp_status run_ln(const void* x, void* h, int64_t n_rows, const dp_blocks* blk, float eps, cudaStream_t s) {
+  cudaError_t e = dp::launch_ln_modulate(x, h, n_rows, blk->hidden, eps, to_table(blk), s);
+  if (e != cudaSuccess) return cuda_fail(e, "ln_modulate launch");
+  return DP_OK;
+}
+
+dp_status run_qkv(const void* h, const void* w_qkv, const float* b_qkv, int64_t n_rows, int32_t hidden, void* q,
+                  void* k, void* v, cudaStream_t s) {
+  dp::GemmArgs g = gemm_args(h, w_qkv, b_qkv, n_rows, 3 * hidden, hidden, dp::kEpiQKV);
+  g.y0 = q;
+  g.y1 = k;
+  g.y2 = v;
+  g.ld_y = hidden;
+  g.seg_cols = hidden;
+  return run_gemm(g, s, "qkv projection launch");
+}
+
+dp_status run_out(const void* o, const void* w_o, const float* b_o, int64_t n_rows, const dp_blocks* blk,
+                  const void* residual, void* out, cudaStream_t s) {
+  dp::GemmArgs g = gemm_args(o, w_o, b_o, n_rows, blk->hidden, blk->hidden, dp::kEpiGateResidual);
+  g.y0 = out;
+  g.ld_y = blk->hidden;
+  g.residual = residual;
+  g.bt = to_table(blk);
+  return run_gemm(g, s, "out projection launch");
+}
+
+}  // namespace
+
+dp_status dp_ln_modulate(const void* x, void* h, int64_t n_rows, const dp_blocks* blk, float eps, void* stream) {
+  dp_status st = check_ln(x, h, n_rows, blk, eps);
+  if (st != DP_OK) return st;
+  return run_ln(x, h, n_rows, blk, eps, static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_linear(const void* a, const void* w, const float* bias, int64_t m, int32_t n, int32_t k, void* y,
+                    dp_dtype y_dt, void* stream) {
+  dp_status st = check_linear(a, w, bias, m, n, k);
+  if (st != DP_OK) return st;
+  if (!y || !aligned16(y)) return fail(DP_ERR_INVALID_ARG, "y NULL or misaligned");
+  if (y_dt != DP_BF16 && y_dt != DP_F16) return fail(DP_ERR_UNSUPPORTED, "y dtype %d (bf16 or f16)", y_dt);
+  if (y == a || y == w) return fail(DP_ERR_INVALID_ARG, "y aliases an input");
+  dp::GemmArgs g = gemm_args(a, w, bias, m, n, k, dp::kEpiStore);
+  g.y0 = y;
+  g.ld_y = n;
+  g.y_f16 = y_dt == DP_F16 ? 1 : 0;
+  return run_gemm(g, static_cast<cudaStream_t>(stream), "linear launch");
+}
+
+dp_status dp_qkv_project(const void* h, const void* w_qkv, const float* b_qkv, int64_t n_rows, int32_t hidden,
+                         void* q, void* k, void* v, void* stream) {
+  if (hidden <= 0 || hidden % 128) return fail(DP_ERR_UNSUPPORTED, "hidden %d (a multiple of 128)", hidden);
+  dp_status st = check_linear(h, w_qkv, b_qkv, n_rows, 3 * static_cast<int64_t>(hidden), hidden);
+  if (st != DP_OK) return st;
+  if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(DP_ERR_INVALID_ARG, "q/k/v NULL or misaligned");
+  if (q == h || k == h || v == h) return fail(DP_ERR_INVALID_ARG, "q/k/v alias h");
+  return run_qkv(h, w_qkv, b_qkv, n_rows, hidden, q, k, v, static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_out_project(const void* o, const void* w_o, const float* b_o, int64_t n_rows, const dp_blocks* blk,
+                         const void* residual, void* out, void* stream) {
+  if (!blk) return fail(DP_ERR_INVALID_ARG, "block table is NULL");
+  const int32_t hidden = blk->hidden;
+  dp_status st = check_linear(o, w_o, b_o, n_rows, hidden, hidden);
+  if (st != DP_OK) return st;
+  st = check_blocks(blk, n_rows, hidden);
+  if (st != DP_OK) return st;
+  if (!residual || !out || !aligned16(residual) || !aligned16(out))
+    return fail(DP_ERR_INVALID_ARG, "residual/out NULL or misaligned");
+  if (out == o || out == w_o || out == residual) return fail(DP_ERR_INVALID_ARG, "out aliases an input");
+  return run_out(o, w_o, b_o, n_rows, blk, residual, out, static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, const void* w_qkv, const float* b_qkv,
+                           const void* w_o, const float* b_o, float eps, dp_kvcache* cache, void* work, void* out,
+                           int32_t n_heads, int32_t head_dim, uint32_t flags, dp_queue* queue,
+                           const void* push_noise, int64_t push_rows, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!cache) return fail(DP_ERR_INVALID_ARG, "cache is NULL");
+  const int64_t hidden64 = static_cast<int64_t>(n_heads) * head_dim;
+  if (n_heads <= 0 || head_dim <= 0 || hidden64 > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_heads/head_dim");
+  const int32_t hidden = static_cast<int32_t>(hidden64);
+  dp_status st = check_ln(x, work, n_win, blk, eps);
+  if (st != DP_OK) return st;
+  if (blk->hidden != hidden) return fail(DP_ERR_INVALID_ARG, "block table hidden %d != %d", blk->hidden, hidden);
+  st = check_linear(x, w_qkv, b_qkv, n_win, 3 * hidden64, hidden);
+  if (st != DP_OK) return st;
+  st = check_linear(x, w_o, b_o, n_win, hidden, hidden);
+  if (st != DP_OK) return st;
+  st = check_cache(cache, hidden, DP_F16);
+  if (st != DP_OK) return st;
+  if (!out || !aligned16(out)) return fail(DP_ERR_INVALID_ARG, "out NULL or misaligned");
+  // work: h (bf16; later the attention output o) | q (bf16) | k (f16) | v (f16), n_win * hidden each
+  const int64_t plane = n_win * hidden64 * 2;
+  char* hw = static_cast<char*>(work);
+  char* qw = hw + plane;
+  char* kw = qw + plane;
+  char* vw = kw + plane;
+  if (out == work || out == x) return fail(DP_ERR_INVALID_ARG, "out aliases x or work");
+  const int64_t rslot = cache_read_slot(cache);
+  const int64_t row_bytes = hidden64 * 2;
+  const char* ck = static_cast<const char*>(cache->k) + rslot * cache->capacity * row_bytes;
+  const char* cv = static_cast<const char*>(cache->v) + rslot * cache->capacity * row_bytes;
+  const int64_t cache_len = cache->len[rslot];
+  st = check_attention(qw, kw, vw, n_win, ck, cv, cache_len, nullptr, hw, n_heads, head_dim, blk, DP_BF16, DP_F16);
+  if (st != DP_OK) return st;
+  const bool pop = (flags & DP_STEP_POP) != 0;
+  const int64_t n_exit = blk->row_offset[1];
+  if (pop && n_exit > cache->capacity)
+    return fail(DP_ERR_CAPACITY, "head block of %lld rows > cache capacity", static_cast<long long>(n_exit));
+  if (queue) {
+    st = check_queue(queue, hidden, DP_BF16);
+    if (st != DP_OK) return st;
+    if (pop && queue->count == 0) return fail(DP_ERR_EMPTY, "pop from an empty queue");
+  }
+  if (push_noise) {
+    if (!queue) return fail(DP_ERR_INVALID_ARG, "push needs a queue");
+    st = check_push(queue, queue->count - (pop ? 1 : 0), push_noise, push_rows);
+    if (st != DP_OK) return st;
+  }
+
+  cudaEvent_t ev[kProfEvents];
+  for (int i = 0; i < kProfEvents; ++i) ev[i] = prof_event(i);
+  cudaError_t e = record(ev[0], s);
+  if (e != cudaSuccess) return cuda_fail(e, "event record");
+  // B1: h = LN(x) * (1 + scale_b) + shift_b
+  st = run_ln(x, hw, n_win, blk, eps, s);
+  if (st != DP_OK) return st;
+  if ((e = record(ev[1], s)) != cudaSuccess) return cuda_fail(e, "event record");
+  // B2: q | k | v = h W_qkv^T + b_qkv
+  st = run_qkv(hw, w_qkv, b_qkv, n_win, hidden, qw, kw, vw, s);
+  if (st != DP_OK) return st;
+  if ((e = record(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event record");
+  // A2: o = attention over [cache ; window] (the modulation already happened before the projection)
+  st = run_attention(qw, kw, vw, n_win, ck, cv, cache_len, nullptr, hw, n_heads, head_dim, 0.0f, blk, 0u, DP_BF16,
+                     DP_F16, s);
+  if (st != DP_OK) return st;
+  if ((e = record(ev[3], s)) != cudaSuccess) return cuda_fail(e, "event record");
+  // B3: out = x + gate_b * (o W_o^T + b_o)
+  st = run_out(hw, w_o, b_o, n_win, blk, x, out, s);
+  if (st != DP_OK) return st;
+  if ((e = record(ev[4], s)) != cudaSuccess) return cuda_fail(e, "event record");
+  // A3: the head block's k, v -> cache ring; noise -> latent ring
+  dp::CopySeg segs[dp::kMaxCopySegs];
+  int nseg = 0;
+  const int64_t wslot = cache->n_advances % cache->n_slots;
+  if (pop) {
+    segs[nseg++] = {kw, static_cast<char*>(cache->k) + wslot * cache->capacity * row_bytes, n_exit * row_bytes};
+    segs[nseg++] = {vw, static_cast<char*>(cache->v) + wslot * cache->capacity * row_bytes, n_exit * row_bytes};
+  }
+  if (push_noise) {
+    const int32_t head_after = (queue->head + (pop ? 1 : 0)) % queue->n_slots;
+    const int32_t count_after = queue->count - (pop ? 1 : 0);
+    const int32_t p = (head_after + count_after) % queue->n_slots;
+    const int64_t bytes = push_rows * row_bytes;
+    segs[nseg++] = {push_noise, queue_slot(queue, p), bytes};
+    segs[nseg++] = {push_noise, queue_slot(queue, p + queue->n_slots), bytes};
+  }
+  if (nseg) {
+    e = dp::launch_copy(segs, nseg, s);
+    if (e != cudaSuccess) return cuda_fail(e, "advance copy");
+  }
+  if ((e = record(ev[5], s)) != cudaSuccess) return cuda_fail(e, "event record");
+  prof_step_done(ev[5], 5);
   if (queue)
     for (int i = 0; i < queue->count; ++i) queue->evals[i] += 1;
   if (pop) {

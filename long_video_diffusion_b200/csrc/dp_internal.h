@@ -69,6 +69,40 @@ cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, 
                             int hidden, const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s);
 cudaError_t launch_copy(const CopySeg* segs, int nseg, cudaStream_t s);
 
+// Linear layer on the tensor cores (dp_gemm.cu): y = a W^T + bias with a [m][k] bf16 and
+// W [n][k] bf16, fp32 accumulation, then one of three epilogues.
+enum GemmEpi {
+  kEpiStore = 0,         // y0 [m][ld_y], bf16 or f16 (y_f16)
+  kEpiQKV = 1,           // columns [0, s) -> y0 (q, bf16), [s, 2s) -> y1 (k, f16), [2s, 3s) -> y2 (v, f16)
+  kEpiGateResidual = 2,  // y0 = residual + gate_b * (a W^T + bias), bf16; b = block of the row
+};
+
+struct GemmArgs {
+  const void* a;
+  const void* w;
+  const float* bias;   // [n] or NULL
+  int64_t m;
+  int32_t n;           // multiple of 128
+  int32_t k;           // multiple of 8
+  int32_t epi;
+  void* y0;
+  void* y1;
+  void* y2;
+  int32_t ld_y;
+  int32_t seg_cols;
+  int32_t y_f16;
+  const void* residual;
+  BlockTable bt;
+  uint32_t* status;
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// Pre-norm and modulation (dp_modulate.cu): h = LN(x) * (1 + scale_b) + shift_b per row,
+// LN without affine over the row's hidden channels in fp32; x and h bf16.
+cudaError_t launch_ln_modulate(const void* x, void* h, int64_t n_rows, int hidden, float eps, const BlockTable& bt,
+                               cudaStream_t s);
+
 // Host-side helper: encode a 2-D 16-bit (f16 or bf16) tensor map [rows][hidden] with a
 // {64 columns, box_rows rows} box and 128-byte swizzle (defined in dp_attn_tc.cu).
 bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, int box_rows, bool f16);

@@ -213,3 +213,39 @@ def test_window_step_checks_before_launch(m):
     q = _queue(m, n_slots=2, slot_rows=128, count=2, rows=(128, 128))
     assert args(0, queue=q, noise=FAKE, rows=128) == m.ERR_CAPACITY  # full queue, no pop
     assert args(m.STEP_POP, queue=_queue(m, count=0)) == m.ERR_EMPTY
+
+
+def test_sublayer_entry_points_check_before_launch(m):
+    P = ctypes.c_void_p
+    blk = _blocks(m, [128, 128], 256)
+    lin = lambda a=FAKE, w=FAKE + 4096, n=256, k=256, y=FAKE + 8192, yd=1, mrows=256: m._lib.dp_linear(
+        P(a), P(w), None, mrows, n, k, P(y), yd, None)
+    assert lin(a=0) == m.ERR_INVALID_ARG
+    assert lin(w=FAKE + 8) == m.ERR_INVALID_ARG                # misaligned
+    assert lin(n=192) == m.ERR_UNSUPPORTED                      # n not a multiple of 128
+    assert lin(k=100) == m.ERR_UNSUPPORTED                      # k not a multiple of 8
+    assert lin(yd=0) == m.ERR_UNSUPPORTED                       # fp32 output
+    assert lin(y=FAKE) == m.ERR_INVALID_ARG                     # y aliases a
+    assert lin(mrows=0) == m.ERR_INVALID_ARG
+    ln = lambda hidden=256, eps=1e-6, rows=(128, 128): m._lib.dp_ln_modulate(
+        P(FAKE), P(FAKE + 4096), sum(rows), ctypes.byref(_blocks(m, list(rows), hidden)), eps, None)
+    assert ln(hidden=128) == m.ERR_UNSUPPORTED                  # hidden not a multiple of 256
+    assert ln(eps=0.0) == m.ERR_INVALID_ARG
+    assert m._lib.dp_ln_modulate(P(FAKE), P(FAKE + 4096), 200, ctypes.byref(blk), 1e-6, None) == m.ERR_INVALID_ARG
+    assert m._lib.dp_qkv_project(P(FAKE), P(FAKE + 4096), None, 256, 192, P(FAKE + 8192), P(FAKE + 16384),
+                                 P(FAKE + 32768), None) == m.ERR_UNSUPPORTED
+    assert m._lib.dp_qkv_project(P(FAKE), P(FAKE + 4096), None, 256, 256, P(FAKE), P(FAKE + 16384),
+                                 P(FAKE + 32768), None) == m.ERR_INVALID_ARG      # q aliases h
+    assert m._lib.dp_out_project(P(FAKE), P(FAKE + 4096), None, 256, ctypes.byref(blk), None, P(FAKE + 8192),
+                                 None) == m.ERR_INVALID_ARG                          # no residual
+    assert m._lib.dp_out_project(P(FAKE), P(FAKE + 4096), None, 256, ctypes.byref(blk), P(FAKE + 16384), P(FAKE),
+                                 None) == m.ERR_INVALID_ARG                          # out aliases o
+    c = _cache(m, capacity=100, hidden=256)
+    step = lambda flags=0, x=FAKE, out=FAKE + (32 << 20), hd=64, queue=None: m._lib.dp_sublayer_step(
+        P(x), 256, ctypes.byref(blk), P(FAKE + (8 << 20)), None, P(FAKE + (16 << 20)), None, 1e-6, ctypes.byref(c),
+        P(FAKE + (64 << 20)), P(out), 256 // hd, hd, flags, ctypes.byref(queue) if queue is not None else None,
+        None, 0, None)
+    assert step(m.STEP_POP) == m.ERR_CAPACITY                  # head block (128 rows) > capacity 100
+    assert c.n_advances == 0
+    assert step(out=FAKE) == m.ERR_INVALID_ARG                  # out aliases x
+    assert step(hd=32) == m.ERR_UNSUPPORTED                     # attention head_dim
