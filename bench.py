@@ -64,6 +64,8 @@ def load_peaks():
 
 def workload(name: str):
     from workloads import step_config
+    if name.startswith("sublayer_"):
+        return step_config(name[len("sublayer_"):])
     if name == "long_run":
         # the oracle arms time a steady-state step of the run (same shapes as its 8-block window)
         return step_config("longrun_steady_bf16")
@@ -371,6 +373,196 @@ def long_run_line(args, world, r):
     }
 
 
+def sublayer_arm(args, rank: int, world: int, local_rank: int):
+    """The DiT attention sublayer step on the window: pre-LN with adaLN modulation, q/k/v
+    projection (tensor cores), window attention over [cache ; window], out projection with
+    the gated residual, and the advance (head block's k, v -> cache, noise pushed)."""
+    import torch
+    import torch.distributed as dist
+
+    import long_video_diffusion_b200 as dp
+    from workloads import as_features, make_step_inputs, make_sublayer_weights
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workload(args.config)
+    x_in = make_step_inputs(cfg)
+    H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
+    wts = {k: t.to(dev) for k, t in make_sublayer_weights(D, cfg.seed + 100).items()}
+    blk = dp.blocks_from_table(x_in["table"].to(dev), x_in["timesteps"], cfg.block_rows)
+    x = x_in["q"].to(dev)
+    noise = x_in["noise"].to(dev)
+    cache = dp.KVCache(cfg.cache_capacity, D, torch.float16,
+                       k=as_features(x_in["cache_k"], cfg.dtype).to(dev).view(1, -1, D),
+                       v=as_features(x_in["cache_v"], cfg.dtype).to(dev).view(1, -1, D), length=cfg.cache_len)
+    queue = dp.Queue(cfg.n_blocks, max(cfg.block_rows), D, device=dev)
+    for _ in range(cfg.n_blocks):
+        dp.queue_push(queue, noise)
+    work = dp.sublayer_work(n, D, device=dev)
+    out = torch.empty(n, D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xx=x, nz=noise):
+        dp.sublayer_step(xx, blk, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], cache, work, out, H, hd,
+                         pop=True, queue=queue, push_noise=nz)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dp.device_status()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(_smi_index(local_rank)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    dp.profile_begin(args.steps)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    stages, _, n_prof = dp.profile_end_stages(5)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    dp.device_status()
+    ms = t0.elapsed_time(t1)
+    stages = [v / n_prof for v in stages]
+
+    hx, hnoise = x_in["q"].pin_memory(), x_in["noise"].pin_memory()
+    hout = torch.empty(n, D, dtype=torch.bfloat16).pin_memory()
+    dx, dnoise = torch.empty_like(x), torch.empty_like(noise)
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        dnoise.copy_(hnoise, non_blocking=True)
+        step(dx, dnoise)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    dp.device_status()
+    vals = max_over_ranks([ms, e2e_ms] + stages, dev)
+    return cfg, dict(ms=vals[0], e2e_ms=vals[1], e2e_steps=e2e_steps, stages=vals[2:], clocks=clocks,
+                     h2d=(hx.numel() + hnoise.numel()) * 2, d2h=hout.numel() * 2)
+
+
+def sublayer_line(args, world, cfg, r):
+    peaks = load_peaks()
+    n, D, H, hd = cfg.n_win, cfg.hidden, cfg.n_heads, cfg.head_dim
+    ln_ms, qkv_ms, attn_ms, out_ms, adv_ms = r["stages"]
+    attn_flop = cfg.attn_flop()
+    qkv_flop = 2 * n * D * 3 * D
+    out_flop = 2 * n * D * D
+    peak = peaks["bf16_tflops_sustained"]
+    tf = lambda flop, ms: flop / (ms / 1e3) / 1e12 if ms > 0 else None
+    achieved = tf(attn_flop, attn_ms)
+    ln_bytes = 2 * n * D * 2
+    adv_bytes = (4 * cfg.block_rows[0] + 3 * cfg.push_rows) * D * 2
+    gbs = lambda b, ms: b / (ms / 1e3) / 1e9 if ms > 0 else None
+    ms_step = r["ms"] / args.steps
+    return {
+        "metric": METRIC, "value": job_throughput(world, n, args.steps, r["ms"]), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "DiT attention sublayer step (pre-LN + adaLN, q/k/v projection, window attention, "
+                               "out projection with gated residual, advance; synthetic weights) on " + describe(cfg),
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": f"inputs larger than L2 (x, W_qkv, W_o {(n * D + 4 * D * D) * 2 / 2**20:.0f} MiB "
+                         f"> {L2_BYTES / 2**20:.0f} MiB)"},
+        "attn_tflops": achieved,
+        "stage_ms": {"ln_modulate": ln_ms, "qkv_projection": qkv_ms, "attention": attn_ms,
+                     "out_projection": out_ms, "advance": adv_ms},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     "traffic_unit": "bytes per launch (see the window-step configurations)",
+                     "kernel": "window_attn_tc_kernel", "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "algorithmic_flop_per_launch": attn_flop},
+        "stage_tensor": {
+            "qkv_projection": {"flop": qkv_flop, "ms": qkv_ms, "achieved_tflops": tf(qkv_flop, qkv_ms),
+                               "frac": (tf(qkv_flop, qkv_ms) or 0) / peak},
+            "out_projection": {"flop": out_flop, "ms": out_ms, "achieved_tflops": tf(out_flop, out_ms),
+                               "frac": (tf(out_flop, out_ms) or 0) / peak}},
+        "stage_hbm": {
+            "ln_modulate": {"bytes": ln_bytes, "ms": ln_ms, "achieved_gbs": gbs(ln_bytes, ln_ms),
+                            "frac": (gbs(ln_bytes, ln_ms) or 0) / peaks["hbm_gbs"]},
+            "advance": {"bytes": adv_bytes, "ms": adv_ms, "achieved_gbs": gbs(adv_bytes, adv_ms),
+                        "frac": (gbs(adv_bytes, adv_ms) or 0) / peaks["hbm_gbs"]}},
+        "clocks": r["clocks"],
+        "e2e": {"value": world * n / (r["e2e_ms"] / r["e2e_steps"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 5 * args.steps,
+    }
+
+
+def oracle_sublayer_sample(cfg, x, wts, n_rows: int, head: int, seed: int):
+    """One oracle sublayer step on a bounded sample: the pre-norm of all rows, the q/k/v
+    projection of all rows for one head's columns, that head's attention for n_rows random
+    query rows, and the out projection of those rows.  Returns (seconds, seconds
+    extrapolated to the whole step): per-head parts times the head count, per-row parts
+    times n_win / n_rows."""
+    import numpy as np
+
+    import oracle as O
+    from workloads import as_features
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(cfg.n_win, size=min(n_rows, cfg.n_win), replace=False))
+    D, hd, H = cfg.hidden, cfg.head_dim, cfg.n_heads
+    c0, c1 = head * hd, (head + 1) * hd
+    mod = O.lookup(x["table"], x["timesteps"])
+    ck = as_features(x["cache_k"], cfg.dtype)[:, c0:c1]
+    cv = as_features(x["cache_v"], cfg.dtype)[:, c0:c1]
+    wq = O.as_f64(wts["w_qkv"])
+    t0 = time.perf_counter()
+    h = O.round_to(O.ln_modulate(x["q"], cfg.row_offset, mod, 1e-6), "bf16")
+    t1 = time.perf_counter()
+    cols = np.concatenate([np.arange(c0, c1), D + np.arange(c0, c1), 2 * D + np.arange(c0, c1)])
+    qkv = O.linear(h, wq[cols], O.as_f64(wts["b_qkv"])[cols])
+    q, k, v = qkv[:, :hd], qkv[:, hd:2 * hd], qkv[:, 2 * hd:]
+    t2 = time.perf_counter()
+    o = O.window_attention(q, k, v, ck, cv, cfg.cache_len, cfg.row_offset, mod[:, :, c0:c1], 1, hd,
+                           mod_q=False, gate_out=False, rows=rows)
+    t3 = time.perf_counter()
+    o_all = np.tile(o, (1, H))
+    O.linear(o_all, wts["w_o"], wts["b_o"])
+    t4 = time.perf_counter()
+    full = (t1 - t0) + (t2 - t1) * H + (t3 - t2) * H * cfg.n_win / len(rows) + (t4 - t3) * cfg.n_win / len(rows)
+    return t4 - t0, full
+
+
+def sublayer_cpu_baseline(cfg, budget_s: float = 12.0):
+    from workloads import make_step_inputs, make_sublayer_weights
+    x = make_step_inputs(cfg)
+    wts = make_sublayer_weights(cfg.hidden, cfg.seed + 100)
+    spent, fulls, i = 0.0, [], 0
+    n_rows = 64
+    while (spent < budget_s or i < 2) and i < 2 * cfg.n_heads:
+        s, full = oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=i)
+        spent += s
+        fulls.append(full)
+        i += 1
+    t = statistics.median(fulls)
+    return {"value": cfg.n_win / t, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"{i} oracle sublayer steps, each: the pre-norm of all {cfg.n_win} rows, the q/k/v projection "
+                       f"of all rows for one head's columns (scaled by {cfg.n_heads} heads), that head's attention for "
+                       f"{n_rows} random rows over all {cfg.cache_len + cfg.n_win} keys and the out projection of those "
+                       f"rows (scaled linearly to all rows); {spent:.1f} s of CPU work")}
+
+
 def stage_hbm(cfg, r, peaks):
     """Achieved HBM bandwidth of the two copy-like stages (algorithmic bytes / event time):
     modulation reads k, v and writes k', v' (4 N_w D e bytes); the advance copies the head
@@ -476,20 +668,26 @@ def cpu_baseline(cfg, budget_s: float = 12.0):
 
 def reference_arm(args):
     """The oracle as the reference arm: W untimed + K timed bounded-sample steps."""
-    from workloads import make_step_inputs
+    from workloads import make_step_inputs, make_sublayer_weights
     cfg = workload(args.config)
     x = make_step_inputs(cfg)
     n_rows = 16
+    if args.config.startswith("sublayer_"):
+        wts = make_sublayer_weights(cfg.hidden, cfg.seed + 100)
+        sample = lambda i, seed: oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=seed)[1]
+        text = "each step: one head's share of an oracle sublayer step (see cpu_baseline of the ours arm)"
+    else:
+        sample = lambda i, seed: oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=seed)[1]
+        text = "each step: " + _sample_text(cfg, n_rows)
     for i in range(args.warmup):
-        oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=1000 + i)
+        sample(i, 1000 + i)
     fulls = []
     for i in range(args.steps):
-        _, full, _ = oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=i)
-        fulls.append(full)
+        fulls.append(sample(i, i))
     ms = 1e3 * statistics.mean(fulls)
     value = cfg.n_win / (ms / 1e3)
     cores = _blas_threads()
-    sample = "each step: " + _sample_text(cfg, n_rows)
+    sample = text
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -539,6 +737,18 @@ def main():
             if not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(workload("long_run"))
                 line["cpu_baseline"]["sample"] = "steady-state step of the run: " + line["cpu_baseline"]["sample"]
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.config.startswith("sublayer_"):
+        cfg, r = sublayer_arm(args, rank, world, local_rank)
+        if rank == 0:
+            line = sublayer_line(args, world, cfg, r)
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = sublayer_cpu_baseline(cfg)
             print(json.dumps(line), flush=True)
         if world > 1:
             import torch.distributed as dist

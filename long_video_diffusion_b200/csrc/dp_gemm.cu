@@ -9,15 +9,22 @@
 //   a: [m][k] bf16 row-major (K contiguous), W: [n][k] bf16 (out-features x in-features,
 //   K contiguous), fp32 accumulation in tensor memory.
 //
-// Design (one CTA = one 128 x BN output tile, BN = 256 or 128):
+// Design: a persistent kernel, one CTA per SM, each walking output tiles of 128 x BN (BN =
+// 256 or 128) in the order tile = blockIdx.x, blockIdx.x + gridDim.x, ...:
 //   warp 0     TMA producer: the A tile (128 x 64) and the W tile (BN x 64) of each K step
-//              (64 bf16 = one 128-byte swizzle row) into a ring of shared-memory stages
-//   warp 1     MMA issuer: four 128 x BN x 16 tcgen05.mma per K step, accumulator in BN
-//              tensor-memory columns; owns the tensor memory
-//   warps 2-5  epilogue: one thread per output row (TMEM lane), 32 columns at a time:
-//              bias, then the variant's store (plain, q/k/v split, gated residual)
-// CTAs walk the n tiles of one m tile consecutively, so W (at most 57 MB here) stays in L2
-// while the A row block is reused from L2 across the n tiles.
+//              (64 bf16 = one 128-byte swizzle row) into a ring of shared-memory stages that
+//              runs on across tiles
+//   warp 1     MMA issuer: four 128 x BN x 16 tcgen05.mma per K step into one of two
+//              tensor-memory accumulators (2 x BN columns), alternating per tile; owns the
+//              tensor memory
+//   warps 2-9  epilogue: two warps per 32-lane quarter of the accumulator, each taking half
+//              of the tile's columns; one thread per output row (TMEM lane), 32 columns at a
+//              time: bias, then the variant's store (plain, q/k/v split, gated residual,
+//              whose residual loads run one chunk ahead); it frees the accumulator for the
+//              tile after next, so a tile's epilogue runs while the next tile's products
+//              accumulate
+// Tiles are numbered m-major (the n tiles of one m tile are consecutive), so the CTAs in
+// flight share a few A row blocks and sweep W, which (at most 57 MB here) stays in L2.
 // Every wait is bounded (dp_device.cuh): on giving up the kernel records a timeout in the
 // device status word, stops, drains its own copies and products, frees TMEM and returns.
 #include <cuda.h>
@@ -41,12 +48,14 @@ struct GemmLayout {
   static constexpr int B_BYTES = BN * GBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-  // full[S], empty[S], acc, fin
-  static constexpr int N_BAR = 2 * STAGES + 2;
+  // full[S], empty[S], acc_full[2], acc_empty[2], fin
+  static constexpr int N_BAR = 2 * STAGES + 5;
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1 KB
-  static constexpr int kThreads = 192;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
   static_assert(ALLOC <= 227 * 1024, "shared memory budget");
   static_assert(BN == 128 || BN == 256, "tile width");
 };
@@ -56,6 +65,7 @@ struct GemmParams {
   int32_t n;
   int32_t k;
   int32_t n_tiles_n;
+  int32_t n_tiles;
   const float* bias;               // [n] or NULL
   void* y0;                        // kEpiStore: y; kEpiQKV: q; kEpiGateResidual: y
   void* y1;                        // kEpiQKV: k
@@ -68,8 +78,16 @@ struct GemmParams {
   BlockTable bt;                   // kEpiGateResidual: gate of the row's block
 };
 
+// The residual of 32 columns of `row` (kEpiGateResidual), as four 16-byte vectors.
+__device__ __forceinline__ void load_res4(const GemmParams& p, int64_t row, int col, uint4 (&r)[4]) {
+  const uint4* src = reinterpret_cast<const uint4*>(p.residual + row * p.n + col);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) r[c] = src[c];
+}
+
 template <int EPI>
-__device__ __forceinline__ void store32(const GemmParams& p, int64_t row, int col, const float (&v)[32]) {
+__device__ __forceinline__ void store32(const GemmParams& p, int64_t row, int col, const float (&v)[32],
+                                        const uint4 (&res)[4]) {
   // v: 32 consecutive output columns col .. col + 31 of `row`, bias already added
   if constexpr (EPI == kEpiStore) {
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y0) + row * p.ld_y + col);
@@ -98,7 +116,6 @@ __device__ __forceinline__ void store32(const GemmParams& p, int64_t row, int co
   } else {
     // y = residual + gate_b * (a W^T + bias), b = block of the row
     const float* gate = block_mod(p.bt, block_of_row(p.bt, row)) + 2 * static_cast<int64_t>(p.n) + col;
-    const uint4* res = reinterpret_cast<const uint4*>(p.residual + row * p.n + col);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.y0) + row * p.ld_y + col);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -141,15 +158,18 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tile = blockIdx.x / p.n_tiles_n;  // consecutive CTAs share the A row block
-  const int n_tile = blockIdx.x % p.n_tiles_n;
   const int KT = (p.k + GBK - 1) / GBK;
+  // this CTA's tiles: blockIdx.x + i * gridDim.x, i < n_mine
+  const int n_mine = p.n_tiles > static_cast<int>(blockIdx.x)
+                         ? (p.n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / gridDim.x
+                         : 0;
 
   const uint32_t bar0 = sb + L::OFF_BAR;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (L::STAGES + s); };
-  const uint32_t acc = bar0 + 8u * (2 * L::STAGES);
-  const uint32_t fin = bar0 + 8u * (2 * L::STAGES + 1);
+  auto acc_full = [&](int b) { return bar0 + 8u * (2 * L::STAGES + b); };
+  auto acc_empty = [&](int b) { return bar0 + 8u * (2 * L::STAGES + 2 + b); };
+  const uint32_t fin = bar0 + 8u * (2 * L::STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -158,13 +178,16 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
-    mbar_init(acc, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 32 * L::kEpiWarps);  // every epilogue thread, after reading the accumulator
+    }
     mbar_init(fin, 1);
     *abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), BN);
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -179,21 +202,29 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % L::STAGES;
-        if (kt >= L::STAGES &&
-            !mbar_wait(empty(s), ((kt / L::STAGES) - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_EMPTY))
-          break;
-        const uint32_t st = sb + s * L::STAGE_BYTES;
-        mbar_arrive_expect_tx(full(s), L::STAGE_BYTES);
-        tma_load_2d(st, &tm_a, kt * GBK, m_tile * GBM, full(s));
-        tma_load_2d(st + L::A_BYTES, &tm_b, kt * GBK, n_tile * BN, full(s));
-        issued = kt + 1;
+      int issued = 0;  // K steps issued over all of this CTA's tiles (the ring's position)
+      bool ok = true;
+      for (int i = 0; ok && i < n_mine; ++i) {
+        const int tile = blockIdx.x + i * gridDim.x;
+        const int m_tile = tile / p.n_tiles_n, n_tile = tile % p.n_tiles_n;
+        for (int kt = 0; kt < KT; ++kt) {
+          const int g = issued;
+          const int s = g % L::STAGES;
+          if (g >= L::STAGES &&
+              !mbar_wait(empty(s), ((g / L::STAGES) - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sb + s * L::STAGE_BYTES;
+          mbar_arrive_expect_tx(full(s), L::STAGE_BYTES);
+          tma_load_2d(st, &tm_a, kt * GBK, m_tile * GBM, full(s));
+          tma_load_2d(st + L::A_BYTES, &tm_b, kt * GBK, n_tile * BN, full(s));
+          issued = g + 1;
+        }
       }
       // every copy this CTA issued lands before its shared memory is released
       const int first = issued > L::STAGES ? issued - L::STAGES : 0;
-      for (int kt = first; kt < issued; ++kt) gemm_drain_wait(full(kt % L::STAGES), (kt / L::STAGES) & 1, p.status);
+      for (int g = first; g < issued; ++g) gemm_drain_wait(full(g % L::STAGES), (g / L::STAGES) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -202,55 +233,83 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       const uint64_t da0 = sdesc_sw128(sb, 16, 1024);
       const uint64_t db0 = sdesc_sw128(sb + L::A_BYTES, 16, 1024);
       bool ok = true;
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % L::STAGES;
-        ok = mbar_wait(full(s), (kt / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV);
-        if (!ok) break;
+      int g = 0;  // K steps consumed (the ring's position)
+      for (int i = 0; ok && i < n_mine; ++i) {
+        const int b = i & 1;
+        // the epilogue has read this accumulator's previous tile (i - 2)
+        if (i >= 2 && !mbar_wait(acc_empty(b), ((i >> 1) - 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O)) break;
         tc_fence_after();
-        const uint64_t so = static_cast<uint64_t>((s * L::STAGE_BYTES) >> 4);
+        const uint32_t d = tmem + static_cast<uint32_t>(b * BN);
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % L::STAGES;
+          ok = mbar_wait(full(s), (g / L::STAGES) & 1, abort, p.status, DEV_ERR_TIMEOUT_KV);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t so = static_cast<uint64_t>((s * L::STAGE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < GBK / 16; ++kk)
-          mma_ss(tmem, da0 + so + kk * 2, db0 + so + kk * 2, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(empty(s));  // the stage is free once these products have read it
+          for (int kk = 0; kk < GBK / 16; ++kk)
+            mma_ss(d, da0 + so + kk * 2, db0 + so + kk * 2, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(empty(s));  // the stage is free once these products have read it
+        }
+        if (ok) mma_commit(acc_full(b));
       }
-      if (ok) mma_commit(acc);
       // every product issued completes before TMEM is released
       mma_commit(fin);
       gemm_drain_wait(fin, 0, p.status);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5)
-    bool ok = mbar_wait(acc, 0, abort, p.status, DEV_ERR_TIMEOUT_O);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    constexpr int kCols = BN / 2;
+    const uint32_t tlane = (static_cast<uint32_t>(quarter) * 32u) << 16;
+    for (int i = 0; i < n_mine; ++i) {
+      const int b = i & 1;
+      bool ok = mbar_wait(acc_full(b), (i >> 1) & 1, abort, p.status, DEV_ERR_TIMEOUT_O);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
       tc_fence_after();
-      const int quarter = warp & 3;  // TMEM lanes this warp may access
+      const int tile = blockIdx.x + i * gridDim.x;
+      const int m_tile = tile / p.n_tiles_n, n_tile = tile % p.n_tiles_n;
       const int64_t row = static_cast<int64_t>(m_tile) * GBM + quarter * 32 + lane;
-      const uint32_t taddr = tmem + ((static_cast<uint32_t>(quarter) * 32u) << 16);
+      const uint32_t taddr = tmem + tlane + static_cast<uint32_t>(b * BN);
+      const bool row_ok = row < p.m;
+      uint4 res_next[4];  // kEpiGateResidual: the next chunk's residual, loaded one chunk ahead
+      if constexpr (EPI == kEpiGateResidual) {
+        if (row_ok) load_res4(p, row, n_tile * BN + half * kCols, res_next);
+      }
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = half * kCols; c0 < (half + 1) * kCols; c0 += 32) {
         const int col = n_tile * BN + c0;
-        if (col >= p.n) break;  // uniform across the CTA
+        uint4 res[4];
+        if constexpr (EPI == kEpiGateResidual) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) res[c] = res_next[c];
+          if (row_ok && c0 + 32 < (half + 1) * kCols) load_res4(p, row, col + 32, res_next);
+        }
         uint32_t r[32];
         tmem_ld32(taddr + c0, r);
         tmem_wait_ld();
-        if (row < p.m) {
+        if (row_ok && col < p.n) {
           float v[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(r[c]);
           if (p.bias) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
-              const float4 b = *reinterpret_cast<const float4*>(p.bias + col + c);
-              v[c] += b.x;
-              v[c + 1] += b.y;
-              v[c + 2] += b.z;
-              v[c + 3] += b.w;
+              const float4 bb = *reinterpret_cast<const float4*>(p.bias + col + c);
+              v[c] += bb.x;
+              v[c + 1] += bb.y;
+              v[c + 2] += bb.z;
+              v[c + 3] += bb.w;
             }
           }
-          store32<EPI>(p, row, col, v);
+          store32<EPI>(p, row, col, v, res);
         }
       }
+      // this thread has read its rows of the accumulator: the MMA may reuse it
+      tc_fence_before();
+      mbar_arrive(acc_empty(b));
     }
   }
 
@@ -258,7 +317,7 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 
@@ -273,6 +332,10 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
   p.n = g.n;
   p.k = g.k;
   p.n_tiles_n = (g.n + BN - 1) / BN;
+  const int64_t m_tiles = (g.m + GBM - 1) / GBM;
+  const int64_t n_tiles = m_tiles * p.n_tiles_n;
+  if (n_tiles > 0x7fffffff) return cudaErrorInvalidValue;
+  p.n_tiles = static_cast<int32_t>(n_tiles);
   p.bias = g.bias;
   p.y0 = g.y0;
   p.y1 = g.y1;
@@ -293,9 +356,10 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int64_t m_tiles = (g.m + GBM - 1) / GBM;
-  const int64_t grid = m_tiles * p.n_tiles_n;
-  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  int sms = 148;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = n_tiles < sms ? n_tiles : sms;  // one resident CTA per SM, each walking tiles
   gemm_tc_kernel<BN, EPI><<<static_cast<unsigned>(grid), L::kThreads, L::ALLOC, s>>>(ta, tb, p);
   return cudaGetLastError();
 }
