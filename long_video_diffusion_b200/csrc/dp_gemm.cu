@@ -23,8 +23,9 @@
 //              whose residual loads run one chunk ahead); it frees the accumulator for the
 //              tile after next, so a tile's epilogue runs while the next tile's products
 //              accumulate
-// Tiles are numbered m-major (the n tiles of one m tile are consecutive), so the CTAs in
-// flight share a few A row blocks and sweep W, which (at most 57 MB here) stays in L2.
+// Tiles are numbered in groups of kGroupM m tiles: within a group the m tiles of one n tile
+// are consecutive, so the ~148 tiles in flight span about 16 row blocks of A and 9 column
+// blocks of W (about 27 MB at hidden 3072) instead of whole rows of W.
 // Every wait is bounded (dp_device.cuh): on giving up the kernel records a timeout in the
 // device status word, stops, drains its own copies and products, frees TMEM and returns.
 #include <cuda.h>
@@ -40,6 +41,18 @@ namespace {
 
 constexpr int GBM = 128;  // output rows per tile
 constexpr int GBK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGroupM = 16;  // m tiles per group of the tile order
+
+// Tile t of the grouped order -> (m tile, n tile).
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles_n, int& m_tile, int& n_tile) {
+  const int per_group = kGroupM * n_tiles_n;
+  const int group = t / per_group;
+  const int first_m = group * kGroupM;
+  const int gm = min(kGroupM, m_tiles - first_m);
+  const int within = t - group * per_group;
+  m_tile = first_m + within % gm;
+  n_tile = within / gm;
+}
 
 template <int BN>
 struct GemmLayout {
@@ -65,6 +78,7 @@ struct GemmParams {
   int32_t n;
   int32_t k;
   int32_t n_tiles_n;
+  int32_t m_tiles;
   int32_t n_tiles;
   const float* bias;               // [n] or NULL
   void* y0;                        // kEpiStore: y; kEpiQKV: q; kEpiGateResidual: y
@@ -205,8 +219,8 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       int issued = 0;  // K steps issued over all of this CTA's tiles (the ring's position)
       bool ok = true;
       for (int i = 0; ok && i < n_mine; ++i) {
-        const int tile = blockIdx.x + i * gridDim.x;
-        const int m_tile = tile / p.n_tiles_n, n_tile = tile % p.n_tiles_n;
+        int m_tile, n_tile;
+        tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, m_tile, n_tile);
         for (int kt = 0; kt < KT; ++kt) {
           const int g = issued;
           const int s = g % L::STAGES;
@@ -269,8 +283,8 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int tile = blockIdx.x + i * gridDim.x;
-      const int m_tile = tile / p.n_tiles_n, n_tile = tile % p.n_tiles_n;
+      int m_tile, n_tile;
+      tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, m_tile, n_tile);
       const int64_t row = static_cast<int64_t>(m_tile) * GBM + quarter * 32 + lane;
       const uint32_t taddr = tmem + tlane + static_cast<uint32_t>(b * BN);
       const bool row_ok = row < p.m;
@@ -335,6 +349,7 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
   const int64_t m_tiles = (g.m + GBM - 1) / GBM;
   const int64_t n_tiles = m_tiles * p.n_tiles_n;
   if (n_tiles > 0x7fffffff) return cudaErrorInvalidValue;
+  p.m_tiles = static_cast<int32_t>(m_tiles);
   p.n_tiles = static_cast<int32_t>(n_tiles);
   p.bias = g.bias;
   p.y0 = g.y0;
