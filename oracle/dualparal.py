@@ -272,10 +272,12 @@ class LongRun:
     steps: the denoiser update needs the trained model, so q = k = v = the block latent).
 
     ``noise``: list of per-block latents (entry order); ``table``: [1000, 3, D];
-    ``tau``: timestep of evaluation index k."""
+    ``tau``: timestep of evaluation index k.  ``context_blocks``: how many of the most
+    recently exited blocks the cache holds and attention reads (1 = the block that just
+    left [R2]; more is the NumC context of several exited blocks)."""
 
     def __init__(self, noise: Sequence, table, n_heads: int, head_dim: int,
-                 window_blocks: int, n_timesteps: int):
+                 window_blocks: int, n_timesteps: int, context_blocks: int = 1):
         self.noise = list(noise)
         self.table = as_f64(table)
         self.n_heads = n_heads
@@ -284,6 +286,7 @@ class LongRun:
         self.T = n_timesteps
         self.tau = timestep_schedule(n_timesteps)
         self.schedule = long_run_schedule(len(self.noise), window_blocks, n_timesteps)
+        self.C = int(context_blocks)
 
     def step_inputs(self, s: int):
         st = self.schedule[s]
@@ -294,16 +297,18 @@ class LongRun:
             ro.append(ro[-1] + a.shape[0])
         t = [self.tau[k] for k in st["k"]]
         mod = lookup(self.table, t)
-        # cache: the most recently exited block's K'/V' from its last evaluation
+        # cache: the K'/V' of the most recently exited block(s), each from its last evaluation
         exited = [b for b in range(len(self.noise))
                   if any(b in self.schedule[u]["pop_after"] for u in range(s))]
         if exited:
-            b = exited[-1]
-            n = as_f64(self.noise[b])
             m_last = lookup(self.table, [self.tau[self.T - 1]])
-            ck = modulate(n, [0, n.shape[0]], m_last)
+            parts = []
+            for b in exited[-self.C:]:
+                n = as_f64(self.noise[b])
+                parts.append(modulate(n, [0, n.shape[0]], m_last))
+            ck = np.concatenate(parts, axis=0)
             cv = ck.copy()
-            L = n.shape[0]
+            L = ck.shape[0]
         else:
             ck = np.zeros((0, x.shape[1]))
             cv = ck

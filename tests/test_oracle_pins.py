@@ -401,3 +401,25 @@ def test_long_run_schedule_golden():
     assert [O.entry_step(b, 50, 8) for b in range(10)] == g["entry_steps_first_10"]
     assert [s["step"] for s in sch if s["pop_after"]][:3] == g["pop_steps_first_3"]
     assert O.timestep_schedule(50)[:5] == g["tau_first_5"]
+
+
+def test_long_run_context_of_several_exited_blocks():
+    """context_blocks = C: the cache is the K'/V' of the last C exited blocks (each modulated at
+    the last timestep); C = 1 is the single exited block of the default run."""
+    rng = np.random.default_rng(5)
+    D, rows = 8, [6, 6, 6, 6, 6, 3]
+    noise = [rng.standard_normal((r, D)) for r in rows]
+    table = np.tanh(rng.standard_normal((1000, 3, D)))
+    one = O.LongRun(noise, table, 2, 4, window_blocks=2, n_timesteps=4)
+    three = O.LongRun(noise, table, 2, 4, window_blocks=2, n_timesteps=4, context_blocks=3)
+    m_last = O.lookup(table, [O.timestep_schedule(4)[3]])
+    for s in range(len(one.schedule)):
+        exited = [b for b in range(len(noise)) if any(b in one.schedule[u]["pop_after"] for u in range(s))]
+        _, _, _, _, ck1, _, L1 = one.step_inputs(s)
+        _, _, _, _, ck3, _, L3 = three.step_inputs(s)
+        assert L1 == (rows[exited[-1]] if exited else 0)
+        assert L3 == sum(rows[b] for b in exited[-3:])
+        want = [O.modulate(noise[b], [0, rows[b]], m_last) for b in exited[-3:]]
+        assert np.array_equal(ck3, np.concatenate(want) if want else np.zeros((0, D)))
+        if exited:
+            assert np.array_equal(ck1, want[-1])
