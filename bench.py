@@ -66,7 +66,7 @@ def workload(name: str):
     from workloads import step_config
     if name.startswith("sublayer_"):
         return step_config(name[len("sublayer_"):])
-    if name == "long_run":
+    if name.startswith("long_run"):
         # the oracle arms time a steady-state step of the run (same shapes as its 8-block window)
         return step_config("longrun_steady_bf16")
     if name.startswith("sweep_"):
@@ -235,7 +235,9 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     timesteps per block): every schedule step is one window step of the library, with the
     window growing from 1 to 8 blocks, the head block exiting into the cache and fresh noise
     blocks pushed.  W warm-up steps run on a separate queue; then the first K schedule steps
-    (all 850 by default) of a fresh run are timed."""
+    (all 850 by default) of a fresh run are timed.  long_run_ctx4: the cache holds the last
+    four exited blocks (8 latent frames, the pages' NumC = 8) and every step attends to all
+    of them."""
     import torch
     import torch.distributed as dist
 
@@ -255,11 +257,18 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     out = torch.empty(n_max, D, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    n_ctx = 4 if args.config == "long_run_ctx4" else 1
+
     def fresh():
-        return dp.KVCache(rc.slot_rows, D, torch.float16, device=dev), dp.Queue(W, rc.slot_rows, D, device=dev)
+        return (dp.KVCache(rc.slot_rows, D, torch.float16, n_slots=n_ctx, device=dev),
+                dp.Queue(W, rc.slot_rows, D, device=dev))
+
+    def cache_rows_read(c):
+        return sum(c.desc.len[i] for i in range(n_ctx)) if n_ctx > 1 else c.length
 
     cache, queue = fresh()
-    dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, max_steps=args.warmup)
+    dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, max_steps=args.warmup,
+                cache_all_slots=n_ctx > 1)
     torch.cuda.synchronize()
     dp.device_status()
 
@@ -273,7 +282,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     def on_step(step, n, popped, pushed):
         steps_n.append(n)
         steps_lc.append(state["lc"])
-        state["lc"] = cache.length
+        state["lc"] = cache_rows_read(cache)
         launches[0] += 2 + (1 if (popped or pushed is not None) else 0)   # modulate, attention (+ copy)
 
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -286,7 +295,8 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         time.sleep(0.3)
     dp.profile_begin(args.steps)
     t0.record(stream)
-    n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps)
+    n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps,
+                          cache_all_slots=n_ctx > 1)
     t1.record(stream)
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
@@ -327,7 +337,8 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps)
+    n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps,
+                        cache_all_slots=n_ctx > 1)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -337,7 +348,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     ms, e2e_ms, attn_ms = max_over_ranks([ms, e2e_ms, attn_ms], dev)
     return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
                 e2e_ms=e2e_ms, e2e_steps=n_e2e, h2d=hb.h2d / max(n_e2e, 1), d2h=d2h[0] / max(n_e2e, 1),
-                clocks=clocks, rc=rc, launches=launches[0])
+                clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx)
 
 
 def long_run_line(args, world, r):
@@ -345,15 +356,15 @@ def long_run_line(args, world, r):
     rc = r["rc"]
     achieved = r["flop"] / (r["attn_ms"] / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    steady_flop = 4 * 21600 * (21600 + 2700) * rc.head_dim * rc.n_heads
+    steady_flop = 4 * 21600 * (21600 + r["n_ctx"] * 2700) * rc.head_dim * rc.n_heads
     return {
         "metric": METRIC, "value": world * r["tokens"] / (r["ms"] / 1e3), "unit": "tokens/s", "n_gpus": world,
         "steps": r["steps"], "warmup": args.warmup, "ms_per_step": r["ms"] / r["steps"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": (f"long_run: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
+        "config": {"workload": (f"{args.config}: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
                                 f"{rc.frames_per_block}-frame blocks, window of {rc.window_blocks} blocks, "
                                 f"{rc.n_timesteps} staggered timesteps per block, {rc.n_heads}x{rc.head_dim} heads, "
-                                f"bf16; first {r['steps']} schedule steps"),
+                                f"bf16, cache of the last {r['n_ctx']} exited block(s); first {r['steps']} schedule steps"),
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "steady-state window q = k = v 66 MiB plus k', v', cache and out: 265 MiB per step > 126 MiB"},
         "window_tokens": r["tokens"],
@@ -727,7 +738,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    if args.config == "long_run":
+    if args.config in ("long_run", "long_run_ctx4"):
         if args.steps == 300 and "--steps" not in sys.argv:
             args.steps = 850                 # the whole run
         r = long_run_arm(args, rank, world, local_rank)

@@ -77,6 +77,10 @@ typedef enum { DP_F32 = 0, DP_BF16 = 1, DP_F16 = 2 } dp_dtype;
 /* dp_window_step flags */
 #define DP_STEP_POP 1u  /* after attention, the head block exits: its K'/V' rows become the
                            cache (and the queue, if given, pops its head) */
+#define DP_STEP_CACHE_ALL_SLOTS 2u  /* attention reads every slot of the cache ring that holds
+                           rows (the K/V of the last n_slots exited blocks: a context of
+                           several blocks, the pages' NumC frames), not only the most
+                           recently written one */
 
 /*
  * Window block table (host plain data, passed by pointer, copied into kernel arguments).
@@ -214,7 +218,9 @@ dp_status dp_queue_pop(dp_queue* q);
  *      rows are written into the cache ring (dp_kvcache_advance), and the queue (if
  *      given) pops its head;
  *   5. if push_noise: it is pushed at the queue's tail (dp_queue_push; needs queue).
- * Steps 4 and 5 run as one copy kernel after the attention on the same stream.  All
+ * With DP_STEP_CACHE_ALL_SLOTS, step 2's cache rows are those of every slot with len > 0
+ * (oldest first; the order does not change the result), else those of the most recently
+ * written slot.  Steps 4 and 5 run as one copy kernel after the attention on the same stream.  All
  * argument checks (including capacities) happen before anything is enqueued.  q, k, v,
  * residual, out, push_noise and the queue are of type dt (bf16 or f32); kv_work and the
  * cache hold features (f16 for bf16, f32 for f32).  q, k and v may alias one another (the

@@ -32,6 +32,7 @@ F32, BF16, F16 = 0, 1, 2
 MOD_Q, GATE_OUT = 1, 2
 TEST_SKIP_KV_LOADS = 0x80000000
 STEP_POP = 1
+STEP_CACHE_ALL_SLOTS = 2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python long_video_diffusion_b200/_build.py` "
@@ -292,10 +293,11 @@ def queue_pop(queue: Queue) -> None:
 
 def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads: int, head_dim: int,
                 pop: bool = False, queue: Optional[Queue] = None, push_noise=None, push_rows=None,
-                residual=None, stream=None, n_win: Optional[int] = None) -> None:
+                residual=None, stream=None, n_win: Optional[int] = None, cache_all_slots: bool = False) -> None:
     """One window step (see dp_window_step).  q, k, v are tensors or raw device addresses
     (n_win then required), e.g. the queue's live window.  kv_work holds at least
-    2 * n_win * hidden feature elements (k' first, v' at element n_win * hidden)."""
+    2 * n_win * hidden feature elements (k' first, v' at element n_win * hidden).
+    cache_all_slots: attend to every cache slot that holds rows (DP_STEP_CACHE_ALL_SLOTS)."""
     if isinstance(q, torch.Tensor):
         ref = q
         n = q.shape[0]
@@ -306,7 +308,8 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
         qp, kp, vp = ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v)
     rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
     _check(_lib.dp_window_step(qp, kp, vp, n, ctypes.byref(blocks), ctypes.byref(cache.desc), _ptr(kv_work),
-                               _ptr(residual), _ptr(out), n_heads, head_dim, STEP_POP if pop else 0,
+                               _ptr(residual), _ptr(out), n_heads, head_dim,
+                               (STEP_POP if pop else 0) | (STEP_CACHE_ALL_SLOTS if cache_all_slots else 0),
                                ctypes.byref(queue.desc) if queue is not None else None, _ptr(push_noise),
                                int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
 
@@ -348,7 +351,8 @@ def sublayer_work(n_win: int, hidden: int, device=None) -> torch.Tensor:
 
 def sublayer_step(x, blocks: DpBlocks, w_qkv, b_qkv, w_o, b_o, cache: KVCache, work, out, n_heads: int,
                   head_dim: int, eps: float = LN_EPS, pop: bool = False, queue: Optional[Queue] = None,
-                  push_noise=None, push_rows=None, stream=None, n_win: Optional[int] = None) -> None:
+                  push_noise=None, push_rows=None, stream=None, n_win: Optional[int] = None,
+                  cache_all_slots: bool = False) -> None:
     """One DiT attention-sublayer step (dp_sublayer_step).  x is a tensor or a raw device
     address (n_win then required), e.g. the queue's live window; work from sublayer_work.
     After the call, work's planes 2 and 3 hold the window's projected k and v (f16)."""
@@ -359,7 +363,8 @@ def sublayer_step(x, blocks: DpBlocks, w_qkv, b_qkv, w_o, b_o, cache: KVCache, w
     rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
     _check(_lib.dp_sublayer_step(xp, n, ctypes.byref(blocks), _ptr(w_qkv), _ptr(b_qkv), _ptr(w_o), _ptr(b_o),
                                  float(eps), ctypes.byref(cache.desc), _ptr(work), _ptr(out), n_heads, head_dim,
-                                 STEP_POP if pop else 0, ctypes.byref(queue.desc) if queue is not None else None,
+                                 (STEP_POP if pop else 0) | (STEP_CACHE_ALL_SLOTS if cache_all_slots else 0),
+                                 ctypes.byref(queue.desc) if queue is not None else None,
                                  _ptr(push_noise), int(rows), _stream(ref, stream)), "dp_sublayer_step")
 
 
@@ -444,13 +449,14 @@ def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
 
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
              queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
-             on_step=None, stream=None, max_steps: Optional[int] = None) -> int:
+             on_step=None, stream=None, max_steps: Optional[int] = None, cache_all_slots: bool = False) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
     noise_blocks: device tensors in entry order.  on_step(step, n_win, popped, pushed) is
     called after each step is enqueued.  max_steps stops the run early (the queue and cache
-    are then left mid-run).  Returns the number of steps."""
+    are then left mid-run).  cache_all_slots: every step attends to all of the cache ring's
+    slots (the last n_slots exited blocks).  Returns the number of steps."""
     T = len(tau)
     n_blocks = len(noise_blocks)
     queue_push(queue, noise_blocks[0], stream=stream)
@@ -461,7 +467,8 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
         pop = queue.evals()[0] + 1 == T
         push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1
         window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,
-                    push_noise=noise_blocks[nxt] if push else None, stream=stream, n_win=n)
+                    push_noise=noise_blocks[nxt] if push else None, stream=stream, n_win=n,
+                    cache_all_slots=cache_all_slots)
         if on_step is not None:
             on_step(step, n, pop, nxt if push else None)
         if push:

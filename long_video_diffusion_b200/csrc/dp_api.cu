@@ -137,6 +137,7 @@ dp_status check_cache(const dp_kvcache* c, int32_t hidden, dp_dtype dt) {
   if (c->hidden != hidden || c->dtype != dt) return fail(DP_ERR_INVALID_ARG, "cache hidden/dtype mismatch");
   if (c->n_slots < 1 || c->n_slots > DP_MAX_SLOTS) return fail(DP_ERR_INVALID_ARG, "cache n_slots %d", c->n_slots);
   if (c->capacity < 0 || c->n_advances < 0) return fail(DP_ERR_INVALID_ARG, "cache capacity/n_advances negative");
+  if (c->capacity * c->n_slots > INT32_MAX) return fail(DP_ERR_CAPACITY, "cache ring rows exceed 2^31 - 1");
   for (int s = 0; s < c->n_slots; ++s)
     if (c->len[s] < 0 || c->len[s] > c->capacity)
       return fail(DP_ERR_CAPACITY, "cache len[%d] = %lld outside [0, capacity]", s, static_cast<long long>(c->len[s]));
@@ -407,10 +408,47 @@ dp_status check_attention(const void* q, const void* k, const void* v, int64_t n
   return check_blocks(blk, n_win, static_cast<int32_t>(hidden));
 }
 
+// A single cache segment: rows [0, cache_len) of cache_k / cache_v.
+dp::CacheSegs one_segment(int64_t cache_len) {
+  dp::CacheSegs g;
+  memset(&g, 0, sizeof(g));
+  g.n = cache_len > 0 ? 1 : 0;
+  g.len[0] = static_cast<int32_t>(cache_len);
+  return g;
+}
+
+// The segments a step reads from the cache ring: the most recently written slot, or with
+// DP_STEP_CACHE_ALL_SLOTS every slot that holds rows, oldest first.  Rows are counted from
+// the ring's base (slot s starts at row s * capacity).
+dp::CacheSegs ring_segments(const dp_kvcache* c, uint32_t flags, int64_t* total) {
+  dp::CacheSegs g;
+  memset(&g, 0, sizeof(g));
+  *total = 0;
+  if (flags & DP_STEP_CACHE_ALL_SLOTS) {
+    for (int i = 0; i < c->n_slots; ++i) {
+      const int64_t slot = (c->n_advances + i) % c->n_slots;  // oldest first
+      if (c->len[slot] <= 0) continue;
+      g.row[g.n] = static_cast<int32_t>(slot * c->capacity);
+      g.len[g.n] = static_cast<int32_t>(c->len[slot]);
+      *total += c->len[slot];
+      g.n += 1;
+    }
+  } else {
+    const int64_t slot = cache_read_slot(c);
+    if (c->len[slot] > 0) {
+      g.n = 1;
+      g.row[0] = static_cast<int32_t>(slot * c->capacity);
+      g.len[0] = static_cast<int32_t>(c->len[slot]);
+      *total = c->len[slot];
+    }
+  }
+  return g;
+}
+
 dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_win, const void* ck, const void* cv,
-                        int64_t cache_len, const void* residual, void* out, int32_t n_heads, int32_t head_dim,
-                        float softmax_scale, const dp_blocks* blk, uint32_t flags, dp_dtype dt, dp_dtype ft,
-                        cudaStream_t s) {
+                        const dp::CacheSegs& segs, int64_t cache_rows, const void* residual, void* out,
+                        int32_t n_heads, int32_t head_dim, float softmax_scale, const dp_blocks* blk, uint32_t flags,
+                        dp_dtype dt, dp_dtype ft, cudaStream_t s) {
   dp::AttnArgs a;
   a.q = q;
   a.k = k;
@@ -420,7 +458,10 @@ dp_status run_attention(const void* q, const void* k, const void* v, int64_t n_w
   a.residual = residual;
   a.out = out;
   a.n_win = n_win;
-  a.cache_len = cache_len;
+  a.cache_len = 0;
+  for (int i = 0; i < segs.n; ++i) a.cache_len += segs.len[i];
+  a.cache_rows = cache_rows;
+  a.segs = segs;
   a.n_heads = n_heads;
   a.head_dim = head_dim;
   a.hidden = n_heads * head_dim;
@@ -443,8 +484,8 @@ dp_status dp_window_attention(const void* q, const void* k, const void* v, int64
   dp_status st =
       check_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, blk, dt, feat_dt);
   if (st != DP_OK) return st;
-  return run_attention(q, k, v, n_win, cache_k, cache_v, cache_len, residual, out, n_heads, head_dim, softmax_scale,
-                       blk, flags, dt, feat_dt, static_cast<cudaStream_t>(stream));
+  return run_attention(q, k, v, n_win, cache_k, cache_v, one_segment(cache_len), cache_len, residual, out, n_heads,
+                       head_dim, softmax_scale, blk, flags, dt, feat_dt, static_cast<cudaStream_t>(stream));
 }
 
 dp_status dp_kvcache_advance(dp_kvcache* c, const void* k_exit, const void* v_exit, int64_t n_exit, void* stream) {
@@ -508,12 +549,13 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   dp_status st = check_cache(cache, hidden, ft);
   if (st != DP_OK) return st;
   if (!kv_work || !aligned16(kv_work)) return fail(DP_ERR_INVALID_ARG, "kv_work NULL or misaligned");
-  const int64_t rslot = cache_read_slot(cache);
   const int64_t row_bytes = hidden64 * elem_bytes(ft);     // features: k', v', cache
   const int64_t in_row_bytes = hidden64 * elem_bytes(dt);  // window inputs and the latent queue
-  const char* ck = static_cast<const char*>(cache->k) + rslot * cache->capacity * row_bytes;
-  const char* cv = static_cast<const char*>(cache->v) + rslot * cache->capacity * row_bytes;
-  const int64_t cache_len = cache->len[rslot];
+  int64_t cache_len = 0;
+  const dp::CacheSegs cseg = ring_segments(cache, flags, &cache_len);
+  const char* ck = static_cast<const char*>(cache->k);
+  const char* cv = static_cast<const char*>(cache->v);
+  const int64_t cache_rows = static_cast<int64_t>(cache->n_slots) * cache->capacity;
   char* kp = static_cast<char*>(kv_work);
   char* vp = kp + n_win * row_bytes;
   st = check_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, blk, dt, ft);
@@ -545,7 +587,7 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
   if (e == cudaSuccess) e = record(ev1, s);
   if (e != cudaSuccess) return cuda_fail(e, "modulate launch");
   // A2: attention with the Q prologue and gate epilogue
-  st = run_attention(q, kp, vp, n_win, ck, cv, cache_len, residual, out, n_heads, head_dim, 0.0f, blk,
+  st = run_attention(q, kp, vp, n_win, ck, cv, cseg, cache_rows, residual, out, n_heads, head_dim, 0.0f, blk,
                      DP_MOD_Q | DP_GATE_OUT, dt, ft, s);
   if (st != DP_OK) return st;
   e = record(ev2, s);
@@ -734,11 +776,12 @@ dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, c
   char* kw = qw + plane;
   char* vw = kw + plane;
   if (out == work || out == x) return fail(DP_ERR_INVALID_ARG, "out aliases x or work");
-  const int64_t rslot = cache_read_slot(cache);
   const int64_t row_bytes = hidden64 * 2;
-  const char* ck = static_cast<const char*>(cache->k) + rslot * cache->capacity * row_bytes;
-  const char* cv = static_cast<const char*>(cache->v) + rslot * cache->capacity * row_bytes;
-  const int64_t cache_len = cache->len[rslot];
+  int64_t cache_len = 0;
+  const dp::CacheSegs cseg = ring_segments(cache, flags, &cache_len);
+  const char* ck = static_cast<const char*>(cache->k);
+  const char* cv = static_cast<const char*>(cache->v);
+  const int64_t cache_rows = static_cast<int64_t>(cache->n_slots) * cache->capacity;
   st = check_attention(qw, kw, vw, n_win, ck, cv, cache_len, nullptr, hw, n_heads, head_dim, blk, DP_BF16, DP_F16);
   if (st != DP_OK) return st;
   const bool pop = (flags & DP_STEP_POP) != 0;
@@ -769,7 +812,7 @@ dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, c
   if (st != DP_OK) return st;
   if ((e = record(ev[2], s)) != cudaSuccess) return cuda_fail(e, "event record");
   // A2: o = attention over [cache ; window] (the modulation already happened before the projection)
-  st = run_attention(qw, kw, vw, n_win, ck, cv, cache_len, nullptr, hw, n_heads, head_dim, 0.0f, blk, 0u, DP_BF16,
+  st = run_attention(qw, kw, vw, n_win, ck, cv, cseg, cache_rows, nullptr, hw, n_heads, head_dim, 0.0f, blk, 0u, DP_BF16,
                      DP_F16, s);
   if (st != DP_OK) return st;
   if ((e = record(ev[3], s)) != cudaSuccess) return cuda_fail(e, "event record");

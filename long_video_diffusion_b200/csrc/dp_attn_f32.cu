@@ -24,7 +24,7 @@ template <int HD>
 __global__ void __launch_bounds__(kRows) attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                                                          const float* __restrict__ v, const float* __restrict__ ck,
                                                          const float* __restrict__ cv, const float* __restrict__ res,
-                                                         float* __restrict__ out, int64_t n_win, int64_t cache_len,
+                                                         float* __restrict__ out, int64_t n_win, CacheSegs segs,
                                                          int hidden, float scale, uint32_t flags, BlockTable bt) {
   __shared__ float sk[kKeys][HD];
   __shared__ float sv[kKeys][HD];
@@ -45,10 +45,13 @@ __global__ void __launch_bounds__(kRows) attn_f32_kernel(const float* __restrict
   }
   float m = -INFINITY, l = 0.0f;
 
-  for (int seg = 0; seg < 2; ++seg) {
-    const float* K = seg == 0 ? ck : k;
-    const float* V = seg == 0 ? cv : v;
-    const int64_t len = seg == 0 ? cache_len : n_win;
+  // the cache segments, then the window
+  for (int seg = 0; seg <= segs.n; ++seg) {
+    const bool in_cache = seg < segs.n;
+    const int64_t base = in_cache ? pick(segs.row, seg) : 0;
+    const float* K = in_cache ? ck + base * hidden : k;
+    const float* V = in_cache ? cv + base * hidden : v;
+    const int64_t len = in_cache ? pick(segs.len, seg) : n_win;
     for (int64_t j0 = 0; j0 < len; j0 += kKeys) {
       const int nk = (len - j0) < kKeys ? static_cast<int>(len - j0) : kKeys;
       __syncthreads();
@@ -95,7 +98,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   attn_f32_kernel<HD><<<grid, kRows, 0, s>>>(
       static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
       static_cast<const float*>(a.cache_k), static_cast<const float*>(a.cache_v), static_cast<const float*>(a.residual),
-      static_cast<float*>(a.out), a.n_win, a.cache_len, a.hidden, a.softmax_scale, a.flags, a.bt);
+      static_cast<float*>(a.out), a.n_win, a.segs, a.hidden, a.softmax_scale, a.flags, a.bt);
   return cudaGetLastError();
 }
 

@@ -33,6 +33,10 @@
 // see PolyPairs); the running max is only moved (and O
 // rescaled) when it grows by more than 2^8, which keeps the result exact because the
 // final 1/l uses the same reference max as the numerator.
+// The cache part of the keys is one contiguous range of rows (the usual case: the block that
+// left) or, in the MULTI instantiation, up to DP_MAX_SLOTS segments of a cache ring (the
+// last exited blocks, read together); the single-range code is kept apart because the
+// softmax loop's instruction schedule is sensitive to any added per-tile work.
 // Every wait is bounded (see dp_device.cuh): on giving up the kernel records a timeout in
 // the device status word, stops issuing work, drains its own copies and MMAs, frees TMEM
 // and returns.
@@ -43,6 +47,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "dp_device.cuh"
@@ -157,6 +162,23 @@ struct Params {
   BlockTable bt;
 };
 
+// Cache segments of the MULTI instantiation: segment s is rows [seg_row[s], seg_row[s] +
+// seg_len[s]) of the cache tensors and key tiles [seg_tile0[s], seg_tile0[s + 1]).
+struct SegParams {
+  int32_t n_seg;
+  int32_t seg_tile0[DP_MAX_SLOTS + 1];
+  int32_t seg_row[DP_MAX_SLOTS];
+  int32_t seg_len[DP_MAX_SLOTS];
+};
+
+// Cache tile j (< the cache tile count) -> its segment: the last s whose first tile is <= j.
+__device__ __forceinline__ int seg_of_tile(const SegParams& sp, int j) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < DP_MAX_SLOTS; ++i) s += (i < sp.n_seg && j >= sp.seg_tile0[i]) ? 1 : 0;
+  return s;
+}
+
 // Bounded wait that ignores the abort flag: used to drain work this CTA already issued.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
   const long long t0 = sm_clock();
@@ -170,11 +192,11 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32
 
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-template <int HD, bool F16>
+template <int HD, bool F16, bool MULTI>
 __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
     window_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                           const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw,
-                          const Params p) {
+                          const Params p, const __grid_constant__ SegParams sp) {
   using L = Layout<HD>;
   constexpr int BN = L::BN;
   constexpr int NQ = L::NQ;
@@ -246,7 +268,13 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
         const bool cache = j < p.n_ct;
         const CUtensorMap* mk = cache ? &tm_kc : &tm_kw;
         const CUtensorMap* mv = cache ? &tm_vc : &tm_vw;
-        const int row = (cache ? j : j - p.n_ct) * BN;
+        int row = (cache ? j : j - p.n_ct) * BN;
+        if constexpr (MULTI) {
+          if (cache) {
+            const int sg = seg_of_tile(sp, j);
+            row = pick(sp.seg_row, sg) + (j - pick(sp.seg_tile0, sg)) * BN;
+          }
+        }
         mbar_arrive_expect_tx(k_full(st), L::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < L::KCH; ++c)
@@ -456,7 +484,13 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
         mbar_arrive(s_free(g));
       }
       const int64_t key0 = (j < p.n_ct) ? static_cast<int64_t>(j) * BN : static_cast<int64_t>(j - p.n_ct) * BN;
-      const int64_t rem = ((j < p.n_ct) ? p.cache_len : p.n_win) - key0;
+      int64_t rem = ((j < p.n_ct) ? p.cache_len : p.n_win) - key0;
+      if constexpr (MULTI) {
+        if (j < p.n_ct) {  // rows left in this tile's segment
+          const int sg = seg_of_tile(sp, j);
+          rem = static_cast<int64_t>(pick(sp.seg_len, sg)) - static_cast<int64_t>(j - pick(sp.seg_tile0, sg)) * BN;
+        }
+      }
       if (rem < BN) {  // last tile of a segment: keys beyond it get -inf (TMA filled them with 0)
         const int valid = static_cast<int>(rem);
 #pragma unroll
@@ -648,20 +682,34 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-template <int HD, bool F16>
+template <int HD, bool F16, bool MULTI>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   using L = Layout<HD>;
   CUtensorMap tkc, tvc, tkw, tvw;
   constexpr int BN = L::BN;
   if (!encode_tmap_16(&tkw, a.k, a.n_win, a.hidden, BN, F16) || !encode_tmap_16(&tvw, a.v, a.n_win, a.hidden, BN, F16))
     return cudaErrorInvalidValue;
+  // one range: the segment's own rows (its first row is the map's row 0); several: the ring
+  const CacheSegs& g = a.segs;
+  const int64_t row_bytes = static_cast<int64_t>(a.hidden) * 2;
+  const char* ck = static_cast<const char*>(a.cache_k) + (MULTI ? 0 : static_cast<int64_t>(g.row[0]) * row_bytes);
+  const char* cv = static_cast<const char*>(a.cache_v) + (MULTI ? 0 : static_cast<int64_t>(g.row[0]) * row_bytes);
+  const int64_t map_rows = MULTI ? a.cache_rows : a.cache_len;
   if (a.cache_len > 0) {
-    if (!encode_tmap_16(&tkc, a.cache_k, a.cache_len, a.hidden, BN, F16) ||
-        !encode_tmap_16(&tvc, a.cache_v, a.cache_len, a.hidden, BN, F16))
+    if (!encode_tmap_16(&tkc, ck, map_rows, a.hidden, BN, F16) || !encode_tmap_16(&tvc, cv, map_rows, a.hidden, BN, F16))
       return cudaErrorInvalidValue;
   } else {
     tkc = tkw;
     tvc = tvw;
+  }
+  SegParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.n_seg = g.n;
+  for (int i = 0; i < DP_MAX_SLOTS; ++i) {
+    const bool in = i < g.n;
+    sp.seg_row[i] = in ? g.row[i] : 0;
+    sp.seg_len[i] = in ? g.len[i] : 0;
+    sp.seg_tile0[i + 1] = sp.seg_tile0[i] + (in ? (g.len[i] + BN - 1) / BN : 0);
   }
   Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -671,7 +719,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   p.cache_len = a.cache_len;
   p.hidden = a.hidden;
   p.n_qpairs = static_cast<int32_t>((a.n_win + L::NQ * BM - 1) / (L::NQ * BM));
-  p.n_ct = static_cast<int32_t>((a.cache_len + BN - 1) / BN);
+  p.n_ct = MULTI ? sp.seg_tile0[DP_MAX_SLOTS] : static_cast<int32_t>((a.cache_len + BN - 1) / BN);
   p.n_wt = static_cast<int32_t>((a.n_win + BN - 1) / BN);
   p.scale_log2 = a.softmax_scale * 1.4426950408889634f;
   p.flags = a.flags;
@@ -683,18 +731,20 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   static bool attr_set[64] = {};  // per instantiation and device
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(window_attn_tc_kernel<HD, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    e = cudaFuncSetAttribute(window_attn_tc_kernel<HD, F16, MULTI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::ALLOC);
     if (e != cudaSuccess) return e;
     // setmaxnreg.inc waits for registers the launch did not provide: refuse to launch if
     // the compiled register count is below the split's assumption.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, window_attn_tc_kernel<HD, F16>);
+    e = cudaFuncGetAttributes(&fa, window_attn_tc_kernel<HD, F16, MULTI>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < L::kLaunchRegs) return cudaErrorInvalidConfiguration;
     attr_set[dev] = true;
   }
   const int64_t grid = static_cast<int64_t>(p.n_qpairs) * a.n_heads;
-  window_attn_tc_kernel<HD, F16><<<static_cast<unsigned>(grid), L::kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw, p);
+  window_attn_tc_kernel<HD, F16, MULTI><<<static_cast<unsigned>(grid), L::kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw,
+                                                                                                  p, sp);
   return cudaGetLastError();
 }
 
@@ -714,8 +764,15 @@ bool encode_tmap_16(void* tmap, const void* base, int64_t rows, int hidden, int 
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, bool f16_features, cudaStream_t s) {
-  if (a.head_dim == 64) return f16_features ? launch_hd<64, true>(a, s) : launch_hd<64, false>(a, s);
-  if (a.head_dim == 128) return f16_features ? launch_hd<128, true>(a, s) : launch_hd<128, false>(a, s);
+  const bool multi = a.segs.n > 1;
+  if (a.head_dim == 64) {
+    if (multi) return f16_features ? launch_hd<64, true, true>(a, s) : launch_hd<64, false, true>(a, s);
+    return f16_features ? launch_hd<64, true, false>(a, s) : launch_hd<64, false, false>(a, s);
+  }
+  if (a.head_dim == 128) {
+    if (multi) return f16_features ? launch_hd<128, true, true>(a, s) : launch_hd<128, false, true>(a, s);
+    return f16_features ? launch_hd<128, true, false>(a, s) : launch_hd<128, false, false>(a, s);
+  }
   return cudaErrorInvalidValue;
 }
 

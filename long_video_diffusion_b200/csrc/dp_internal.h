@@ -32,6 +32,24 @@ __host__ __device__ __forceinline__ const float* block_mod(const BlockTable& t, 
   return m;
 }
 
+// The cache rows attention reads: segment s is rows [row[s], row[s] + len[s]) of cache_k /
+// cache_v (one segment per cache slot read; zero segments when the cache is empty).
+struct CacheSegs {
+  int32_t n;
+  int32_t row[DP_MAX_SLOTS];
+  int32_t len[DP_MAX_SLOTS];
+};
+
+// Element i of a small kernel-argument array, selected with compile-time indices (a run-time
+// index into a kernel argument would copy it to local memory).
+template <int N>
+__host__ __device__ __forceinline__ int32_t pick(const int32_t (&a)[N], int i) {
+  int32_t v = a[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k) v = (k == i) ? a[k] : v;
+  return v;
+}
+
 struct AttnArgs {
   const void* q;
   const void* k;
@@ -41,7 +59,9 @@ struct AttnArgs {
   const void* residual;
   void* out;
   int64_t n_win;
-  int64_t cache_len;
+  int64_t cache_len;    // total cache rows read (the sum of the segments' lengths)
+  int64_t cache_rows;   // rows cache_k / cache_v hold (the extent the segments index into)
+  CacheSegs segs;
   int32_t n_heads;
   int32_t head_dim;
   int32_t hidden;
