@@ -35,13 +35,19 @@ Parity status of each function (how it is pinned, in tests/test_oracle_pins.py):
   round_to          pinned: hand-computed bf16/f16 bit patterns, f16 saturation
   sublayer_step     pinned: identity projections reduce it to x + gated window_attention
                     of the normed window; brute-force loops end to end on tiny inputs
+  coordinated_frames / coordinated_schedule / gather_frames
+                    pinned: a hand-worked selection; first window = the pool in order;
+                    later blocks distinct, disjoint from the previous block, in permutation
+                    order; gathered rows equal the pool's frames
 """
 from .dualparal import (as_f64, row_blocks, lookup, modulate, modulate_rounded,
                         window_attention, window_step, KVCacheRing, FifoQueue,
                         entry_step, long_run_schedule, timestep_schedule, LongRun)
 from .sublayer import round_to, layer_norm, ln_modulate, linear, sublayer_step
+from .noise_init import coordinated_frames, coordinated_schedule, gather_frames
 
 __all__ = ["as_f64", "row_blocks", "lookup", "modulate", "modulate_rounded",
            "window_attention", "window_step", "KVCacheRing", "FifoQueue", "entry_step",
            "long_run_schedule", "timestep_schedule", "LongRun", "round_to", "layer_norm",
-           "ln_modulate", "linear", "sublayer_step"]
+           "ln_modulate", "linear", "sublayer_step", "coordinated_frames",
+           "coordinated_schedule", "gather_frames"]

@@ -85,3 +85,18 @@ def make_sublayer_weights(hidden: int, seed: int) -> Dict[str, torch.Tensor]:
     w_o = _randn(g, (hidden, hidden), s).to(torch.bfloat16).contiguous()
     b_o = _randn(g, (hidden,), 0.02).contiguous()
     return {"w_qkv": w_qkv, "b_qkv": b_qkv, "w_o": w_o, "b_o": b_o}
+
+
+def make_noise_permutations(n_blocks: int, pool_frames: int, seed: int) -> List[List[int]]:
+    """One seeded random permutation of the noise pool's frames per block (the random draw of
+    the coordinated noise initialisation, an input to both sides)."""
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randperm(pool_frames, generator=g).tolist() for _ in range(n_blocks)]
+
+
+def make_run_pool(cfg: RunConfig, dtype: str = "bf16") -> torch.Tensor:
+    """The noise pool of the long run with coordinated initialisation: the first window's
+    noise, [window_blocks * frames_per_block, frame_rows, hidden], drawn after the table."""
+    g = torch.Generator().manual_seed(cfg.seed + 1000)
+    n = cfg.window_blocks * cfg.frames_per_block
+    return to_dtype(_randn(g, (n, cfg.frame_rows, cfg.hidden)), dtype)
