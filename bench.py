@@ -33,8 +33,8 @@ METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 
 # DRAM bytes (read + write) of one attention launch from an ncu capture (summaries under
 # profiles/), valid only for the kernel source they were captured on (md5 over
 # csrc/dp_attn_tc.cu and csrc/dp_device.cuh); any other source reports null.
-TRAFFIC_SOURCE_MD5 = "021dac6c4a1364996dd7c7e37e5b6f2e"
-TRAFFIC_BYTES = {"cogvideo_bf16": 232.533504e6 + 50.983424e6, "wan_bf16": 630.609152e6 + 142.060032e6}
+TRAFFIC_SOURCE_MD5 = "4c480125da97a60609b40285a9993232"
+TRAFFIC_BYTES = {"cogvideo_bf16": 232.779776e6 + 51.218176e6, "wan_bf16": 629.861376e6 + 141.78688e6}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -237,12 +237,13 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     blocks pushed.  W warm-up steps run on a separate queue; then the first K schedule steps
     (all 850 by default) of a fresh run are timed.  long_run_ctx4: the cache holds the last
     four exited blocks (8 latent frames, the pages' NumC = 8) and every step attends to all
-    of them."""
+    of them.  long_run_coord: blocks are pushed with the coordinated noise initialisation
+    (frames of a pool holding the first window's noise, in a fresh random order per block)."""
     import torch
     import torch.distributed as dist
 
     import long_video_diffusion_b200 as dp
-    from workloads import make_run_noise, make_run_table, run_config
+    from workloads import make_noise_permutations, make_run_noise, make_run_pool, make_run_table, run_config
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -258,6 +259,15 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     stream = torch.cuda.current_stream(dev)
 
     n_ctx = 4 if args.config == "long_run_ctx4" else 1
+    frame_pool = None
+    if args.config == "long_run_coord":
+        pool = make_run_pool(rc).to(dev)
+        nf = [r // rc.frame_rows for r in rc.block_rows]
+        perms = make_noise_permutations(len(nf), pool.shape[0], seed=rc.seed + 2000)
+        lists = [list(range(b * rc.frames_per_block, (b + 1) * rc.frames_per_block)) for b in range(W)]
+        for b in range(W, len(nf)):
+            lists.append(dp.coordinated_frames(pool.shape[0], nf[b], lists[b - 1], perms[b]))
+        frame_pool = (pool, lists)
 
     def fresh():
         return (dp.KVCache(rc.slot_rows, D, torch.float16, n_slots=n_ctx, device=dev),
@@ -268,7 +278,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
 
     cache, queue = fresh()
     dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, max_steps=args.warmup,
-                cache_all_slots=n_ctx > 1)
+                cache_all_slots=n_ctx > 1, frame_pool=frame_pool)
     torch.cuda.synchronize()
     dp.device_status()
 
@@ -283,7 +293,10 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         steps_n.append(n)
         steps_lc.append(state["lc"])
         state["lc"] = cache_rows_read(cache)
-        launches[0] += 2 + (1 if (popped or pushed is not None) else 0)   # modulate, attention (+ copy)
+        if frame_pool is None:   # modulate, attention (+ one copy for the pop and the push)
+            launches[0] += 2 + (1 if (popped or pushed is not None) else 0)
+        else:                    # modulate, attention (+ the pop's copy) (+ the push's gather)
+            launches[0] += 2 + (1 if popped else 0) + (1 if pushed is not None else 0)
 
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(_smi_index(local_rank)) if rank == 0 else None
@@ -296,7 +309,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     dp.profile_begin(args.steps)
     t0.record(stream)
     n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps,
-                          cache_all_slots=n_ctx > 1)
+                          cache_all_slots=n_ctx > 1, frame_pool=frame_pool)
     t1.record(stream)
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
@@ -332,13 +345,21 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         d2h[0] += n * D * 2
 
     cache, queue = fresh()
+    e2e_pool = None
+    if frame_pool is not None:   # the pool is the run's input: copied from pinned host memory once
+        hpool = frame_pool[0].cpu().pin_memory()
+        dpool = torch.empty_like(frame_pool[0])
+        hb.h2d = hpool.numel() * 2
+        e2e_pool = (dpool, frame_pool[1])
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    if e2e_pool is not None:
+        e2e_pool[0].copy_(hpool, non_blocking=True)
     n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps,
-                        cache_all_slots=n_ctx > 1)
+                        cache_all_slots=n_ctx > 1, frame_pool=e2e_pool)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -738,7 +759,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    if args.config in ("long_run", "long_run_ctx4"):
+    if args.config in ("long_run", "long_run_ctx4", "long_run_coord"):
         if args.steps == 300 and "--steps" not in sys.argv:
             args.steps = 850                 # the whole run
         r = long_run_arm(args, rank, world, local_rank)

@@ -204,6 +204,19 @@ dp_status dp_kvcache_advance(dp_kvcache* c, const void* k_exit, const void* v_ex
  * slot_rows; INVALID_ARG if the current tail is a short (final) block. */
 dp_status dp_queue_push(dp_queue* q, const void* noise, int64_t rows, void* stream);
 
+/* Coordinated noise initialisation's push (the abstract: initial noise patterns shared
+ * without extra cost; the review: each new block drawn from the full noise space, shuffled so
+ * that concatenated blocks do not repeat noise): the pushed block is the concatenation of
+ * frames frame_idx[0 .. n_frames) (host array) of pool (DEVICE [pool_frames][frame_rows]
+ * [hidden], the queue's type), written to the queue's tail slot like dp_queue_push (byte
+ * copy, bit-exact).  Which frames (the shuffle) is the caller's choice; the binding's
+ * coordinated_frames() implements the selection rule.  n_frames in [1, 16] (UNSUPPORTED
+ * otherwise); INVALID_ARG for an index outside [0, pool_frames); CAPACITY as dp_queue_push
+ * for n_frames * frame_rows rows. */
+dp_status dp_queue_push_frames(dp_queue* q, const void* pool, int32_t pool_frames,
+                               int64_t frame_rows, const int32_t* frame_idx, int32_t n_frames,
+                               void* stream);
+
 /* Pop the head block (metadata only: the slot becomes free).  EMPTY if no block. */
 dp_status dp_queue_pop(dp_queue* q);
 

@@ -77,6 +77,7 @@ _SIGS = {
     "dp_kvcache_advance": [ctypes.POINTER(DpKvcache), _P, _P, _I64, _P],
     "dp_queue_push": [ctypes.POINTER(DpQueue), _P, _I64, _P],
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
+    "dp_queue_push_frames": [ctypes.POINTER(DpQueue), _P, _I32, _I64, ctypes.POINTER(_I32), _I32, _P],
     "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
     "dp_window_step_noalloc": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P,
@@ -287,6 +288,28 @@ def queue_push(queue: Queue, noise: torch.Tensor, rows: Optional[int] = None, st
            "dp_queue_push")
 
 
+def queue_push_frames(queue: Queue, pool: torch.Tensor, frames: Sequence[int], stream=None) -> None:
+    """Push a block made of pool frames (dp_queue_push_frames); pool [frames][frame_rows][hidden]."""
+    idx = (_I32 * len(frames))(*[int(f) for f in frames])
+    _check(_lib.dp_queue_push_frames(ctypes.byref(queue.desc), _ptr(pool), pool.shape[0], pool.shape[1], idx,
+                                     len(frames), _stream(queue.latent, stream)), "dp_queue_push_frames")
+
+
+def coordinated_frames(pool_frames: int, block_frames: int, prev_frames: Sequence[int],
+                       perm: Sequence[int]) -> list:
+    """Frames of a new block under the coordinated noise initialisation: the pool's frames in
+    the order of the random permutation perm, without the frames the previous block used
+    (adjacent blocks share no noise frame), the first block_frames of them."""
+    prev = set(int(f) for f in prev_frames)
+    out = []
+    for f in perm:
+        if int(f) not in prev:
+            out.append(int(f))
+            if len(out) == block_frames:
+                return out
+    raise ValueError("the pool has too few frames outside the previous block")
+
+
 def queue_pop(queue: Queue) -> None:
     _check(_lib.dp_queue_pop(ctypes.byref(queue.desc)), "dp_queue_pop")
 
@@ -449,26 +472,38 @@ def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
 
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
              queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
-             on_step=None, stream=None, max_steps: Optional[int] = None, cache_all_slots: bool = False) -> int:
+             on_step=None, stream=None, max_steps: Optional[int] = None, cache_all_slots: bool = False,
+             frame_pool=None) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
     noise_blocks: device tensors in entry order.  on_step(step, n_win, popped, pushed) is
     called after each step is enqueued.  max_steps stops the run early (the queue and cache
     are then left mid-run).  cache_all_slots: every step attends to all of the cache ring's
-    slots (the last n_slots exited blocks).  Returns the number of steps."""
+    slots (the last n_slots exited blocks).  frame_pool = (pool, frame_lists): blocks are
+    pushed as pool frames (dp_queue_push_frames; the coordinated noise initialisation) and
+    noise_blocks only gives each block's row count.  Returns the number of steps."""
     T = len(tau)
     n_blocks = len(noise_blocks)
-    queue_push(queue, noise_blocks[0], stream=stream)
+    def push_block(b):
+        if frame_pool is None:
+            queue_push(queue, noise_blocks[b], stream=stream)
+        else:
+            queue_push_frames(queue, frame_pool[0], frame_pool[1][b], stream=stream)
+
+    push_block(0)
     nxt = 1
     step = 0
     while queue.count > 0 and (max_steps is None or step < max_steps):
         blk, win, n = queue_blocks(queue, table, tau)
         pop = queue.evals()[0] + 1 == T
         push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1
+        fused_push = push and frame_pool is None
         window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,
-                    push_noise=noise_blocks[nxt] if push else None, stream=stream, n_win=n,
+                    push_noise=noise_blocks[nxt] if fused_push else None, stream=stream, n_win=n,
                     cache_all_slots=cache_all_slots)
+        if push and not fused_push:
+            push_block(nxt)
         if on_step is not None:
             on_step(step, n, pop, nxt if push else None)
         if push:

@@ -526,6 +526,38 @@ dp_status dp_queue_push(dp_queue* q, const void* noise, int64_t rows, void* stre
   return DP_OK;
 }
 
+dp_status dp_queue_push_frames(dp_queue* q, const void* pool, int32_t pool_frames, int64_t frame_rows,
+                               const int32_t* frame_idx, int32_t n_frames, void* stream) {
+  if (!q) return fail(DP_ERR_INVALID_ARG, "queue is NULL");
+  dp_status st = check_queue(q, q->hidden, q->dtype);
+  if (st != DP_OK) return st;
+  if (!frame_idx) return fail(DP_ERR_INVALID_ARG, "frame_idx is NULL");
+  if (n_frames < 1 || n_frames > dp::kMaxGatherFrames)
+    return fail(DP_ERR_UNSUPPORTED, "n_frames %d outside [1, %d]", n_frames, dp::kMaxGatherFrames);
+  if (pool_frames < 1 || frame_rows < 1) return fail(DP_ERR_INVALID_ARG, "pool_frames/frame_rows");
+  for (int i = 0; i < n_frames; ++i)
+    if (frame_idx[i] < 0 || frame_idx[i] >= pool_frames)
+      return fail(DP_ERR_INVALID_ARG, "frame_idx[%d] = %d outside [0, %d)", i, frame_idx[i], pool_frames);
+  const int64_t rows = frame_rows * n_frames;
+  st = check_push(q, q->count, pool, rows);
+  if (st != DP_OK) return st;
+  const int64_t frame_bytes = frame_rows * q->hidden * elem_bytes(q->dtype);
+  if (frame_bytes % 16 || frame_bytes / 16 > UINT32_MAX) return fail(DP_ERR_INVALID_ARG, "frame size");
+  const int32_t p = (q->head + q->count) % q->n_slots;
+  dp::FrameGather g;
+  memset(&g, 0, sizeof(g));
+  g.pool = static_cast<const uint4*>(pool);
+  g.dst0 = static_cast<uint4*>(static_cast<void*>(queue_slot(q, p)));
+  g.dst1 = static_cast<uint4*>(static_cast<void*>(queue_slot(q, p + q->n_slots)));
+  g.vec_per_frame = static_cast<uint32_t>(frame_bytes / 16);
+  g.n_frames = n_frames;
+  for (int i = 0; i < n_frames; ++i) g.idx[i] = frame_idx[i];
+  cudaError_t e = dp::launch_gather_frames(g, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "frame gather");
+  apply_push(q, rows);
+  return DP_OK;
+}
+
 dp_status dp_queue_pop(dp_queue* q) {
   if (!q) return fail(DP_ERR_INVALID_ARG, "queue is NULL");
   dp_status st = check_queue(q, q->hidden, q->dtype);

@@ -3,6 +3,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <vector_types.h>
 
 #include "dp.h"
 
@@ -88,6 +89,19 @@ dp_status set_error(dp_status s, const char* msg);
 cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, int64_t n_rows,
                             int hidden, const BlockTable& bt, dp_dtype x_dt, dp_dtype y_dt, cudaStream_t s);
 cudaError_t launch_copy(const CopySeg* segs, int nseg, cudaStream_t s);
+
+// Frames idx[0 .. n_frames) of a pool ([frames][vec_per_frame] 16-byte vectors) copied in that
+// order to dst0 and to dst1 (a queue slot and its mirror).
+constexpr int kMaxGatherFrames = 16;
+struct FrameGather {
+  const uint4* pool;
+  uint4* dst0;
+  uint4* dst1;
+  uint32_t vec_per_frame;
+  int32_t n_frames;
+  int32_t idx[kMaxGatherFrames];
+};
+cudaError_t launch_gather_frames(const FrameGather& g, cudaStream_t s);
 
 // Linear layer on the tensor cores (dp_gemm.cu): y = a W^T + bias with a [m][k] bf16 and
 // W [n][k] bf16, fp32 accumulation, then one of three epilogues.

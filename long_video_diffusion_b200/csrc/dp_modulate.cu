@@ -216,6 +216,22 @@ __global__ void __launch_bounds__(kThreads) copy_kernel(CopySegs segs) {
   }
 }
 
+// Gather of whole latent frames from a noise pool into a queue slot and its mirror (the
+// coordinated noise initialisation's push: each new block is a shuffled selection of the
+// pool's frames).  grid.y = output frame; byte copy, bit-exact.
+__global__ void __launch_bounds__(kThreads) gather_frames_kernel(FrameGather g) {
+  const int f = blockIdx.y;
+  const uint4* src = g.pool + static_cast<size_t>(pick(g.idx, f)) * g.vec_per_frame;
+  uint4* d0 = g.dst0 + static_cast<size_t>(f) * g.vec_per_frame;
+  uint4* d1 = g.dst1 + static_cast<size_t>(f) * g.vec_per_frame;
+  const uint32_t stride = gridDim.x * kThreads;
+  for (uint32_t i = blockIdx.x * kThreads + threadIdx.x; i < g.vec_per_frame; i += stride) {
+    const uint4 v = __ldcs(src + i);
+    d0[i] = v;
+    d1[i] = v;
+  }
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -271,6 +287,16 @@ cudaError_t launch_ln_modulate(const void* x, void* h, int64_t n_rows, int hidde
   else
     ln_modulate_kernel<kLnMaxVec><<<static_cast<unsigned>(grid), 32 * kLnWarps, 0, s>>>(
         static_cast<const uint4*>(x), static_cast<uint4*>(h), static_cast<uint32_t>(n_rows), hidden, eps, bt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_frames(const FrameGather& g, cudaStream_t s) {
+  if (g.n_frames < 1 || g.n_frames > kMaxGatherFrames || g.vec_per_frame == 0) return cudaErrorInvalidValue;
+  const uint64_t per_frame = (static_cast<uint64_t>(g.vec_per_frame) + kThreads * kUnroll - 1) / (kThreads * kUnroll);
+  const uint64_t cap = (static_cast<uint64_t>(sm_count()) * 8 + g.n_frames - 1) / g.n_frames;
+  dim3 grid(static_cast<unsigned>(per_frame < cap ? (per_frame > 0 ? per_frame : 1) : cap),
+            static_cast<unsigned>(g.n_frames));
+  gather_frames_kernel<<<grid, kThreads, 0, s>>>(g);
   return cudaGetLastError();
 }
 
