@@ -115,50 +115,41 @@ __global__ void __launch_bounds__(1024) modulate_kernel(const uint4* __restrict_
 
 // Pre-norm and modulation of the DiT attention sublayer (adaLN: the block's shift and scale
 // applied to the layer-normed hidden state): h = (x - mean) / sqrt(var + eps) * (1 + scale_b)
-// + shift_b, mean and var over the row's channels in fp32 (two passes over the row held in
-// registers), rounded once to bf16.  One warp per row; lane l holds the row's 16-byte
-// vectors l, l + 32, ...; hidden is a multiple of 256 and at most 32 * 256.
-constexpr int kLnMaxVec = 32;
+// + shift_b, mean and var over the row's channels in fp32 (two passes), rounded once to
+// bf16.  One warp per row; lane l handles the row's 16-byte vectors l, l + 32, ...  The row
+// is read three times (sum, squared deviations, output) rather than held in registers: the
+// second and third reads hit L1/L2, and the few registers leave room for 64 warps per SM,
+// which is what hides the memory latency of a one-row-per-warp reduction.
 constexpr int kLnWarps = 8;
 
-// kMaxVec: the most 16-byte vectors a lane holds (hidden <= kMaxVec * 256); 16 keeps two CTAs
-// resident per SM for hidden up to 4096.
-template <int kMaxVec>
 __global__ void __launch_bounds__(32 * kLnWarps) ln_modulate_kernel(const uint4* __restrict__ x, uint4* __restrict__ h,
                                                                    uint32_t n_rows, int hidden, float eps,
                                                                    BlockTable bt) {
   const int lane = threadIdx.x & 31;
   const uint32_t row = blockIdx.x * kLnWarps + (threadIdx.x >> 5);
   if (row >= n_rows) return;
-  const int vpr = hidden / 8;          // 16-byte vectors per row
-  const int vpl = vpr / 32;            // per lane
+  const int vpr = hidden / 8;  // 16-byte vectors per row
   const uint4* xr = x + static_cast<size_t>(row) * vpr;
-  uint4 v[kMaxVec];
   float sum = 0.0f;
+#pragma unroll 4
+  for (int i = lane; i < vpr; i += 32) {
+    float f[8];
+    unpack8<kBF16>(__ldg(xr + i), f);
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    if (i < vpl) {
-      v[i] = __ldcs(xr + i * 32 + lane);
-      float f[8];
-      unpack8<kBF16>(v[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sum += f[e];
-    }
+    for (int e = 0; e < 8; ++e) sum += f[e];
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float mean = sum / static_cast<float>(hidden);
   float sq = 0.0f;
+#pragma unroll 4
+  for (int i = lane; i < vpr; i += 32) {
+    float f[8];
+    unpack8<kBF16>(__ldg(xr + i), f);
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    if (i < vpl) {
-      float f[8];
-      unpack8<kBF16>(v[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = f[e] - mean;
-        sq = fmaf(d, d, sq);
-      }
+    for (int e = 0; e < 8; ++e) {
+      const float d = f[e] - mean;
+      sq = fmaf(d, d, sq);
     }
   }
 #pragma unroll
@@ -166,22 +157,20 @@ __global__ void __launch_bounds__(32 * kLnWarps) ln_modulate_kernel(const uint4*
   const float rstd = 1.0f / sqrtf(sq / static_cast<float>(hidden) + eps);
   const float* m = block_mod(bt, block_of_row(bt, row));
   uint4* hr = h + static_cast<size_t>(row) * vpr;
+#pragma unroll 2
+  for (int i = lane; i < vpr; i += 32) {
+    const int col = i * 8;
+    float f[8];
+    unpack8<kBF16>(__ldg(xr + i), f);
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(m + col));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(m + col + 4));
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(m + hidden + col));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(m + hidden + col + 4));
+    const float sh[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    if (i < vpl) {
-      const int col = (i * 32 + lane) * 8;
-      float f[8];
-      unpack8<kBF16>(v[i], f);
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(m + col));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(m + col + 4));
-      const float4 c0 = __ldg(reinterpret_cast<const float4*>(m + hidden + col));
-      const float4 c1 = __ldg(reinterpret_cast<const float4*>(m + hidden + col + 4));
-      const float sh[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = fmaf((f[e] - mean) * rstd, 1.0f + sc[e], sh[e]);
-      hr[i * 32 + lane] = pack8<kBF16>(f);
-    }
+    for (int e = 0; e < 8; ++e) f[e] = fmaf((f[e] - mean) * rstd, 1.0f + sc[e], sh[e]);
+    __stcs(hr + i, pack8<kBF16>(f));
   }
 }
 
@@ -279,14 +268,10 @@ cudaError_t launch_modulate(const void* const* src, void* const* dst, int nseg, 
 
 cudaError_t launch_ln_modulate(const void* x, void* h, int64_t n_rows, int hidden, float eps, const BlockTable& bt,
                                cudaStream_t s) {
-  if (n_rows <= 0 || n_rows >= (1ll << 31) || hidden % 256 || hidden > kLnMaxVec * 256) return cudaErrorInvalidValue;
+  if (n_rows <= 0 || n_rows >= (1ll << 31) || hidden % 256 || hidden > 8192) return cudaErrorInvalidValue;
   const uint64_t grid = (static_cast<uint64_t>(n_rows) + kLnWarps - 1) / kLnWarps;
-  if (hidden <= 16 * 256)
-    ln_modulate_kernel<16><<<static_cast<unsigned>(grid), 32 * kLnWarps, 0, s>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(h), static_cast<uint32_t>(n_rows), hidden, eps, bt);
-  else
-    ln_modulate_kernel<kLnMaxVec><<<static_cast<unsigned>(grid), 32 * kLnWarps, 0, s>>>(
-        static_cast<const uint4*>(x), static_cast<uint4*>(h), static_cast<uint32_t>(n_rows), hidden, eps, bt);
+  ln_modulate_kernel<<<static_cast<unsigned>(grid), 32 * kLnWarps, 0, s>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(h), static_cast<uint32_t>(n_rows), hidden, eps, bt);
   return cudaGetLastError();
 }
 
