@@ -73,15 +73,15 @@ constexpr float kPolyC2 = 0.2426111251115799f;
 constexpr float kPolyC3 = 0.0551716685295105f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer
 constexpr float kPolyMinX = -125.0f;
-// Column pairs (of the 16 in each 32-column chunk) whose exponentials use the polynomial,
-// spread evenly over the chunk: 6 of 16 at head_dim 64 and 4 of 16 at head_dim 128 (measured
-// best among 0, 3, 4, 6, 8, 10 and 12 of 16; more moves the limit to the issue slots and the
-// FMA pipe, where the polynomial costs about seven instructions a pair against one MUFU
-// instruction per exponential).  Head_dim 128 has half the exponentials per product, so the
-// MUFU unit is less of a limit there.
+// Column pairs (of the 16 in each 32-column chunk) whose exponentials use the polynomial: 4
+// of 16, spread over the chunk (measured best among 0, 3, 4, 5, 6, 8, 10 and 12 of 16; more
+// moves the limit to the issue slots and the FMA pipe, where the polynomial costs about
+// seven instructions a pair against one MUFU instruction per exponential).  Where they sit
+// changes the compiler's interleaving of the two kinds: at head_dim 64, pairs 0, 5, 10, 15
+// ran 3-4 % faster than 0, 4, 8, 12 and than the earlier 6 of 16 (1, 4, 6, 9, 11, 14).
 template <int HD>
 struct PolyPairs {
-  static constexpr uint32_t kMask = HD == 64 ? 0x4A52u : 0x1111u;
+  static constexpr uint32_t kMask = HD == 64 ? 0x8421u : 0x1111u;
 };
 
 template <int HD>
