@@ -13,7 +13,7 @@ Sources (page title, then the part of it):
   [R3] same review, supporting citation of DiT-style conditioning (the model is a
        Diffusion Transformer whose blocks are conditioned on their own timestep).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * adaLN modulation is y = x * (1 + scale_b) + shift_b, per channel, with (shift, scale,
     gate) the rows of a per-timestep table; the gate multiplies the attention output.
   * q, k and v of the window are modulated with their own block's vectors; cached K/V are

@@ -10,7 +10,7 @@ Sources (page title, then the part of it):
        patterns; the recipe is a full noise pool, shuffled assignment and the exclusion of
        the last few latents.
 
-Reading where the pages are silent (also listed in the design doc): the pool is the initial
+Reading where the pages are silent: the pool is the initial
 noise of the first window, one independent N(0, 1) draw per latent frame; the first
 window's blocks take the pool's frames in order; every later block takes its frames from
 the pool in the order of a fresh random permutation, skipping the frames of the block just

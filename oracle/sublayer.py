@@ -10,7 +10,7 @@ Sources (page title, then the part of it):
   [R3] same review, supporting citations: DiT-style conditioning of every block on its own
        timestep.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * the sublayer is the DiT self-attention sublayer with adaLN conditioning:
         h   = LN(x) * (1 + scale_b) + shift_b          (LN without affine parameters)
         q, k, v = h W_qkv^T + b_qkv                     (W: out-features x in-features)
