@@ -179,17 +179,6 @@ __device__ __forceinline__ int seg_of_tile(const SegParams& sp, int j) {
   return s;
 }
 
-// Bounded wait that ignores the abort flag: used to drain work this CTA already issued.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
-  const long long t0 = sm_clock();
-  while (!mbar_try_wait(bar, parity)) {
-    if (sm_clock() - t0 > kWaitLimitCycles) {
-      atomicOr(status, DEV_ERR_TIMEOUT_DRAIN);
-      return;
-    }
-  }
-}
-
 __device__ __forceinline__ float4 ld_f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 template <int HD, bool F16, bool MULTI>
@@ -288,8 +277,8 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
       // every copy this CTA issued must land before its shared memory is released
       const int first = issued > L::STAGES ? issued - L::STAGES : 0;
       for (int j = first; j < issued; ++j) {
-        drain_wait(k_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
-        drain_wait(v_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
+        mbar_drain_wait(k_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
+        mbar_drain_wait(v_full(j % L::STAGES), (j / L::STAGES) & 1, p.status);
       }
     }
   } else if (lane == 0) {
@@ -408,7 +397,7 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
     if (warp >= L::W_ISS) {
       // every product this warp issued completes before TMEM is released
       mma_commit(fin);
-      drain_wait(fin, 0, p.status);
+      mbar_drain_wait(fin, 0, p.status);
     }
   }
   } else {

@@ -120,6 +120,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait that ignores the abort flag, for draining work the caller already issued
+// (its own TMA copies or MMAs) before shared or tensor memory is released: gives up after
+// kWaitLimitCycles and records DEV_ERR_TIMEOUT_DRAIN.
+__device__ __forceinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
+  const long long t0 = sm_clock();
+  while (!mbar_try_wait(bar, parity)) {
+    if (sm_clock() - t0 > kWaitLimitCycles) {
+      atomicOr(status, DEV_ERR_TIMEOUT_DRAIN);
+      return;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

@@ -151,17 +151,6 @@ __device__ __forceinline__ void store32(const GemmParams& p, int64_t row, int co
   }
 }
 
-// Bounded wait that ignores the abort flag: used to drain work this CTA already issued.
-__device__ __forceinline__ void gemm_drain_wait(uint32_t bar, uint32_t parity, uint32_t* status) {
-  const long long t0 = sm_clock();
-  while (!mbar_try_wait(bar, parity)) {
-    if (sm_clock() - t0 > kWaitLimitCycles) {
-      atomicOr(status, DEV_ERR_TIMEOUT_DRAIN);
-      return;
-    }
-  }
-}
-
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -238,7 +227,7 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       }
       // every copy this CTA issued lands before its shared memory is released
       const int first = issued > L::STAGES ? issued - L::STAGES : 0;
-      for (int g = first; g < issued; ++g) gemm_drain_wait(full(g % L::STAGES), (g / L::STAGES) & 1, p.status);
+      for (int g = first; g < issued; ++g) mbar_drain_wait(full(g % L::STAGES), (g / L::STAGES) & 1, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -269,7 +258,7 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       }
       // every product issued completes before TMEM is released
       mma_commit(fin);
-      gemm_drain_wait(fin, 0, p.status);
+      mbar_drain_wait(fin, 0, p.status);
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9)
