@@ -193,32 +193,30 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     ms = t0.elapsed_time(t1)
     attn_ms, mod_ms, adv_ms = attn_ms / n_prof, mod_ms / n_prof, adv_ms / n_prof
 
-    # ---- e2e: the same step through the public API with pinned host buffers
+    # ---- e2e: the same step through the public API from pinned host buffers, every step's
+    # inputs copied in and its output read back inside the timed region (the library's
+    # StepPipeline overlaps step i's copies with step i - 1's compute on three streams)
     hq, hk, hv = (x[key].pin_memory() for key in ("q", "k", "v"))
     hnoise = x["noise"].pin_memory()
     hout = torch.empty(n, D, dtype=torch.bfloat16).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dnoise = torch.empty_like(noise)
     e2e_steps = max(3, min(args.steps, 50))
+    pipe = dp.StepPipeline(n, D, noise.shape[0], device=dev)
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dnoise.copy_(hnoise, non_blocking=True)
-        dp.window_step(dq, dk, dv, blk, cache, kv, out, H, hd, pop=True, queue=queue, push_noise=dnoise)
-        hout.copy_(out, non_blocking=True)
+        pipe.submit(hq, hk, hv, hnoise, hout, blk, cache, kv, H, hd, pop=True, queue=queue)
 
     for _ in range(3):
         e2e_step()
+    pipe.finish()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(pipe.h2d)
     for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
+    e1.record(pipe.d2h)
+    pipe.finish()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     dp.device_status()

@@ -337,6 +337,65 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
                                int(rows), _dtype(out), _stream(ref, stream)), "dp_window_step")
 
 
+# ------------------------------------------------------------------------- host-fed steps
+
+class StepPipeline:
+    """Window steps fed from host memory with the copies overlapped with the compute.
+
+    Step i's inputs (q, k, v and the noise block, from pinned host tensors) are copied on a
+    copy stream into one of ``depth`` device buffer sets while step i - 1 computes on the
+    compute stream, and step i - 1's output is read back on a third stream while step i
+    computes.  Events order the three: a buffer set is refilled only after the step that
+    used it has finished computing, and the output buffer only after its read-back.  Each
+    step is one dp_window_step on the compute stream; queue and cache descriptors advance in
+    submission order as usual.  finish() waits for everything submitted."""
+
+    def __init__(self, n_win: int, hidden: int, noise_rows: int, dtype=torch.bfloat16, depth: int = 2,
+                 device=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.depth = depth
+        mk = lambda rows: [torch.empty(rows, hidden, dtype=dtype, device=dev) for _ in range(depth)]
+        self.q, self.k, self.v, self.out = mk(n_win), mk(n_win), mk(n_win), mk(n_win)
+        self.noise = mk(noise_rows)
+        self.h2d = torch.cuda.Stream(dev)
+        self.compute = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.copied, self.computed, self.read = ev(), ev(), ev()
+        self.n = 0
+
+    def submit(self, hq, hk, hv, hnoise, hout, blocks: DpBlocks, cache: KVCache, kv_work, n_heads: int,
+               head_dim: int, pop: bool = True, queue: Optional[Queue] = None) -> None:
+        """Enqueue one step: host inputs hq, hk, hv, hnoise (pinned), host output hout."""
+        i = self.n % self.depth
+        with torch.cuda.stream(self.h2d):
+            if self.n >= self.depth:
+                self.h2d.wait_event(self.computed[i])      # the step that used buffer set i is done
+            self.q[i].copy_(hq, non_blocking=True)
+            self.k[i].copy_(hk, non_blocking=True)
+            self.v[i].copy_(hv, non_blocking=True)
+            if hnoise is not None:
+                self.noise[i][:hnoise.shape[0]].copy_(hnoise, non_blocking=True)
+            self.copied[i].record(self.h2d)
+        self.compute.wait_event(self.copied[i])
+        if self.n >= self.depth:
+            self.compute.wait_event(self.read[i])          # out[i] has been read back
+        window_step(self.q[i], self.k[i], self.v[i], blocks, cache, kv_work, self.out[i], n_heads, head_dim,
+                    pop=pop, queue=queue, push_noise=None if hnoise is None else self.noise[i][:hnoise.shape[0]],
+                    stream=self.compute)
+        self.computed[i].record(self.compute)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.computed[i])
+            hout.copy_(self.out[i], non_blocking=True)
+            self.read[i].record(self.d2h)
+        self.n += 1
+
+    def finish(self) -> None:
+        for s in (self.h2d, self.compute, self.d2h):
+            s.synchronize()
+
+
 # ------------------------------------------------------------------------- B: DiT attention sublayer
 
 LN_EPS = 1e-6
