@@ -340,24 +340,28 @@ def window_step(q, k, v, blocks: DpBlocks, cache: KVCache, kv_work, out, n_heads
 # ------------------------------------------------------------------------- host-fed steps
 
 class StepPipeline:
-    """Window steps fed from host memory with the copies overlapped with the compute.
+    """Steps fed from host memory with the copies overlapped with the compute.
 
-    Step i's inputs (q, k, v and the noise block, from pinned host tensors) are copied on a
-    copy stream into one of ``depth`` device buffer sets while step i - 1 computes on the
-    compute stream, and step i - 1's output is read back on a third stream while step i
-    computes.  Events order the three: a buffer set is refilled only after the step that
-    used it has finished computing, and the output buffer only after its read-back.  Each
-    step is one dp_window_step on the compute stream; queue and cache descriptors advance in
-    submission order as usual.  finish() waits for everything submitted."""
+    Step i's inputs (pinned host tensors) are copied on a copy stream into one of ``depth``
+    device buffer sets while step i - 1 computes on the compute stream, and step i - 1's
+    output is read back on a third stream while step i computes.  Events order the three: a
+    buffer set is refilled only after the step that used it has finished computing, and the
+    output buffer only after its read-back.  Queue and cache descriptors advance in
+    submission order as usual.  finish() waits for everything submitted.
+
+    shapes: the device shapes of the step's inputs, in the order submit_with() receives them
+    (for submit(): q, k, v and the noise block); out_shape: the step's output."""
 
     def __init__(self, n_win: int, hidden: int, noise_rows: int, dtype=torch.bfloat16, depth: int = 2,
-                 device=None):
+                 device=None, shapes=None, out_shape=None):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.device = dev
         self.depth = depth
-        mk = lambda rows: [torch.empty(rows, hidden, dtype=dtype, device=dev) for _ in range(depth)]
-        self.q, self.k, self.v, self.out = mk(n_win), mk(n_win), mk(n_win), mk(n_win)
-        self.noise = mk(noise_rows)
+        if shapes is None:
+            shapes = [(n_win, hidden)] * 3 + [(noise_rows, hidden)]
+        out_shape = out_shape or (n_win, hidden)
+        self.inputs = [[torch.empty(*sh, dtype=dtype, device=dev) for sh in shapes] for _ in range(depth)]
+        self.out = [torch.empty(*out_shape, dtype=dtype, device=dev) for _ in range(depth)]
         self.h2d = torch.cuda.Stream(dev)
         self.compute = torch.cuda.Stream(dev)
         self.d2h = torch.cuda.Stream(dev)
@@ -365,31 +369,40 @@ class StepPipeline:
         self.copied, self.computed, self.read = ev(), ev(), ev()
         self.n = 0
 
-    def submit(self, hq, hk, hv, hnoise, hout, blocks: DpBlocks, cache: KVCache, kv_work, n_heads: int,
-               head_dim: int, pop: bool = True, queue: Optional[Queue] = None) -> None:
-        """Enqueue one step: host inputs hq, hk, hv, hnoise (pinned), host output hout."""
+    def submit_with(self, host_inputs, hout, run) -> None:
+        """Enqueue one step: copy host_inputs (pinned; None entries are skipped) into a device
+        buffer set, call run(device_inputs, device_out, compute_stream) to enqueue the step's
+        work, and read device_out back into hout."""
         i = self.n % self.depth
+        dins = self.inputs[i]
         with torch.cuda.stream(self.h2d):
             if self.n >= self.depth:
                 self.h2d.wait_event(self.computed[i])      # the step that used buffer set i is done
-            self.q[i].copy_(hq, non_blocking=True)
-            self.k[i].copy_(hk, non_blocking=True)
-            self.v[i].copy_(hv, non_blocking=True)
-            if hnoise is not None:
-                self.noise[i][:hnoise.shape[0]].copy_(hnoise, non_blocking=True)
+            for d, h in zip(dins, host_inputs):
+                if h is not None:
+                    d[:h.shape[0]].copy_(h, non_blocking=True)
             self.copied[i].record(self.h2d)
         self.compute.wait_event(self.copied[i])
         if self.n >= self.depth:
             self.compute.wait_event(self.read[i])          # out[i] has been read back
-        window_step(self.q[i], self.k[i], self.v[i], blocks, cache, kv_work, self.out[i], n_heads, head_dim,
-                    pop=pop, queue=queue, push_noise=None if hnoise is None else self.noise[i][:hnoise.shape[0]],
-                    stream=self.compute)
+        run(dins, self.out[i], self.compute)
         self.computed[i].record(self.compute)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.computed[i])
-            hout.copy_(self.out[i], non_blocking=True)
+            hout.copy_(self.out[i][:hout.shape[0]], non_blocking=True)
             self.read[i].record(self.d2h)
         self.n += 1
+
+    def submit(self, hq, hk, hv, hnoise, hout, blocks: DpBlocks, cache: KVCache, kv_work, n_heads: int,
+               head_dim: int, pop: bool = True, queue: Optional[Queue] = None) -> None:
+        """One window step (dp_window_step) on host inputs hq, hk, hv, hnoise (pinned; hnoise may
+        be None), its output read back into hout."""
+        rows = None if hnoise is None else hnoise.shape[0]
+
+        def run(d, out, stream):
+            window_step(d[0], d[1], d[2], blocks, cache, kv_work, out, n_heads, head_dim, pop=pop, queue=queue,
+                        push_noise=None if rows is None else d[3][:rows], stream=stream)
+        self.submit_with([hq, hk, hv, hnoise], hout, run)
 
     def finish(self) -> None:
         for s in (self.h2d, self.compute, self.d2h):
