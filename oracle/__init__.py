@@ -35,6 +35,11 @@ Parity status of each function (how it is pinned, in tests/test_oracle_pins.py):
   round_to          pinned: hand-computed bf16/f16 bit patterns, f16 saturation
   sublayer_step     pinned: identity projections reduce it to x + gated window_attention
                     of the normed window; brute-force loops end to end on tiny inputs
+  fresh_context / fresh_context_sublayer
+                    pinned: equal to the window step's and the sublayer step's own
+                    features of the same rows; zero shift/scale -> the rows; a
+                    hand-computed LN + projection; the long run's cache at its final
+                    timestep
   coordinated_frames / coordinated_schedule / gather_frames
                     pinned: a hand-worked selection; first window = the pool in order;
                     later blocks distinct, disjoint from the previous block, in permutation
@@ -45,9 +50,11 @@ from .dualparal import (as_f64, row_blocks, lookup, modulate, modulate_rounded,
                         entry_step, long_run_schedule, timestep_schedule, LongRun)
 from .sublayer import round_to, layer_norm, ln_modulate, linear, sublayer_step
 from .noise_init import coordinated_frames, coordinated_schedule, gather_frames
+from .context import fresh_context, fresh_context_sublayer
 
 __all__ = ["as_f64", "row_blocks", "lookup", "modulate", "modulate_rounded",
            "window_attention", "window_step", "KVCacheRing", "FifoQueue", "entry_step",
            "long_run_schedule", "timestep_schedule", "LongRun", "round_to", "layer_norm",
            "ln_modulate", "linear", "sublayer_step", "coordinated_frames",
-           "coordinated_schedule", "gather_frames"]
+           "coordinated_schedule", "gather_frames", "fresh_context",
+           "fresh_context_sublayer"]
