@@ -64,6 +64,8 @@ def load_peaks():
 
 def workload(name: str):
     from workloads import step_config
+    if name.startswith("sublayer_fresh_"):
+        return step_config(name[len("sublayer_fresh_"):])
     if name.startswith("sublayer_"):
         return step_config(name[len("sublayer_"):])
     if name.startswith("long_run"):
@@ -406,7 +408,10 @@ def long_run_line(args, world, r):
 def sublayer_arm(args, rank: int, world: int, local_rank: int):
     """The DiT attention sublayer step on the window: pre-LN with adaLN modulation, q/k/v
     projection (tensor cores), window attention over [cache ; window], out projection with
-    the gated residual, and the advance (head block's k, v -> cache, noise pushed)."""
+    the gated residual, and the advance (head block's k, v -> cache, noise pushed).  The
+    ``sublayer_fresh_*`` workloads recompute the context's k, v before every step (pre-LN of
+    the context rows conditioned on timestep 0, then the k/v projection) instead of reusing
+    the cached ones: the cost side of the cache's staleness ablation."""
     import torch
     import torch.distributed as dist
 
@@ -431,8 +436,24 @@ def sublayer_arm(args, rank: int, world: int, local_rank: int):
     work = dp.sublayer_work(n, D, device=dev)
     out = torch.empty(n, D, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    fresh = args.config.startswith("sublayer_fresh_")
+    n_ctx = cfg.cache_len
+    x_ctx = x[:n_ctx].clone()                 # the context block's rows, resident like the cache
+    ctx_blk = dp.blocks_from_table(x_in["table"].to(dev), [0], [n_ctx])
+    ref_ev = []
 
-    def step(xx=x, nz=noise):
+    def refresh(strm=None, timed=False):
+        if timed:
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            e[0].record(stream)
+        dp.context_refresh_sublayer(x_ctx, ctx_blk, wts["w_qkv"], wts["b_qkv"], cache, work, stream=strm)
+        if timed:
+            e[1].record(stream)
+            ref_ev.append(e)
+
+    def step(xx=x, nz=noise, timed=False):
+        if fresh:
+            refresh(timed=timed)
         dp.sublayer_step(xx, blk, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], cache, work, out, H, hd,
                          pop=True, queue=queue, push_noise=nz)
 
@@ -451,10 +472,11 @@ def sublayer_arm(args, rank: int, world: int, local_rank: int):
     dp.profile_begin(args.steps)
     t0.record(stream)
     for _ in range(args.steps):
-        step()
+        step(timed=True)
     t1.record(stream)
     torch.cuda.synchronize()
     stages, _, n_prof = dp.profile_end_stages(5)
+    refresh_ms = sum(a.elapsed_time(b) for a, b in ref_ev) / len(ref_ev) if ref_ev else None
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()
@@ -470,6 +492,8 @@ def sublayer_arm(args, rank: int, world: int, local_rank: int):
     pipe = dp.StepPipeline(n, D, noise.shape[0], device=dev, shapes=[(n, D), tuple(noise.shape)])
 
     def run(d, dout, strm):
+        if fresh:
+            refresh(strm)
         dp.sublayer_step(d[0], blk, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], cache, work, dout, H, hd,
                          pop=True, queue=queue, push_noise=d[1], stream=strm)
 
@@ -491,9 +515,12 @@ def sublayer_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     dp.device_status()
-    vals = max_over_ranks([ms, e2e_ms] + stages, dev)
+    vals = max_over_ranks([ms, e2e_ms] + stages + [refresh_ms or 0.0], dev)
+    refresh_ms = vals[-1] if fresh else None
+    vals = vals[:-1]
     return cfg, dict(ms=vals[0], e2e_ms=vals[1], e2e_steps=e2e_steps, stages=vals[2:], clocks=clocks,
-                     h2d=(hx.numel() + hnoise.numel()) * 2, d2h=hout.numel() * 2)
+                     h2d=(hx.numel() + hnoise.numel()) * 2, d2h=hout.numel() * 2,
+                     refresh_ms=refresh_ms, n_ctx=n_ctx if fresh else 0)
 
 
 def sublayer_line(args, world, cfg, r):
@@ -510,12 +537,16 @@ def sublayer_line(args, world, cfg, r):
     adv_bytes = (4 * cfg.block_rows[0] + 3 * cfg.push_rows) * D * 2
     gbs = lambda b, ms: b / (ms / 1e3) / 1e9 if ms > 0 else None
     ms_step = r["ms"] / args.steps
-    return {
+    n_ctx = r["n_ctx"]
+    fresh_text = (f"; context k, v recomputed before every step (pre-LN + k/v projection of {n_ctx} context rows)"
+                  if n_ctx else "")
+    line = {
         "metric": METRIC, "value": job_throughput(world, n, args.steps, r["ms"]), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "DiT attention sublayer step (pre-LN + adaLN, q/k/v projection, window attention, "
-                               "out projection with gated residual, advance; synthetic weights) on " + describe(cfg),
+                               "out projection with gated residual, advance; synthetic weights) on " + describe(cfg)
+                               + fresh_text,
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": f"inputs larger than L2 (x, W_qkv, W_o {(n * D + 4 * D * D) * 2 / 2**20:.0f} MiB "
                          f"> {L2_BYTES / 2**20:.0f} MiB)"},
@@ -540,16 +571,27 @@ def sublayer_line(args, world, cfg, r):
         "clocks": r["clocks"],
         "e2e": {"value": world * n / (r["e2e_ms"] / r["e2e_steps"] / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (7 if n_ctx else 5) * args.steps,
     }
+    if n_ctx:
+        kv_flop = 2 * n_ctx * D * 2 * D
+        ref_ms = r["refresh_ms"]
+        line["stage_ms"]["context_refresh"] = ref_ms
+        line["stage_tensor"]["context_refresh"] = {
+            "flop": kv_flop, "ms": ref_ms, "achieved_tflops": tf(kv_flop, ref_ms),
+            "frac": (tf(kv_flop, ref_ms) or 0) / peak,
+            "note": "pre-LN of the context rows plus their k/v projection, timed together"}
+    return line
 
 
-def oracle_sublayer_sample(cfg, x, wts, n_rows: int, head: int, seed: int):
+def oracle_sublayer_sample(cfg, x, wts, n_rows: int, head: int, seed: int, fresh: bool = False):
     """One oracle sublayer step on a bounded sample: the pre-norm of all rows, the q/k/v
     projection of all rows for one head's columns, that head's attention for n_rows random
     query rows, and the out projection of those rows.  Returns (seconds, seconds
     extrapolated to the whole step): per-head parts times the head count, per-row parts
-    times n_win / n_rows."""
+    times n_win / n_rows.  ``fresh``: the context's k, v are first recomputed whole (pre-norm
+    and k/v projection of the context rows, conditioned on timestep 0) and the attention
+    reads them."""
     import numpy as np
 
     import oracle as O
@@ -562,6 +604,14 @@ def oracle_sublayer_sample(cfg, x, wts, n_rows: int, head: int, seed: int):
     ck = as_features(x["cache_k"], cfg.dtype)[:, c0:c1]
     cv = as_features(x["cache_v"], cfg.dtype)[:, c0:c1]
     wq = O.as_f64(wts["w_qkv"])
+    t_ctx = 0.0
+    if fresh:
+        tc = time.perf_counter()
+        n_ctx = cfg.cache_len
+        fk, fv = O.fresh_context_sublayer(x["q"][:n_ctx], [0, n_ctx], O.lookup(x["table"], [0]), wts["w_qkv"],
+                                          wts["b_qkv"], 1e-6)
+        ck, cv = fk[:, c0:c1], fv[:, c0:c1]
+        t_ctx = time.perf_counter() - tc
     t0 = time.perf_counter()
     h = O.round_to(O.ln_modulate(x["q"], cfg.row_offset, mod, 1e-6), "bf16")
     t1 = time.perf_counter()
@@ -576,17 +626,17 @@ def oracle_sublayer_sample(cfg, x, wts, n_rows: int, head: int, seed: int):
     O.linear(o_all, wts["w_o"], wts["b_o"])
     t4 = time.perf_counter()
     full = (t1 - t0) + (t2 - t1) * H + (t3 - t2) * H * cfg.n_win / len(rows) + (t4 - t3) * cfg.n_win / len(rows)
-    return t4 - t0, full
+    return t4 - t0 + t_ctx, full + t_ctx
 
 
-def sublayer_cpu_baseline(cfg, budget_s: float = 12.0):
+def sublayer_cpu_baseline(cfg, budget_s: float = 12.0, fresh: bool = False):
     from workloads import make_step_inputs, make_sublayer_weights
     x = make_step_inputs(cfg)
     wts = make_sublayer_weights(cfg.hidden, cfg.seed + 100)
     spent, fulls, i = 0.0, [], 0
     n_rows = 64
     while (spent < budget_s or i < 2) and i < 2 * cfg.n_heads:
-        s, full = oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=i)
+        s, full = oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=i, fresh=fresh)
         spent += s
         fulls.append(full)
         i += 1
@@ -595,7 +645,9 @@ def sublayer_cpu_baseline(cfg, budget_s: float = 12.0):
             "sample": (f"{i} oracle sublayer steps, each: the pre-norm of all {cfg.n_win} rows, the q/k/v projection "
                        f"of all rows for one head's columns (scaled by {cfg.n_heads} heads), that head's attention for "
                        f"{n_rows} random rows over all {cfg.cache_len + cfg.n_win} keys and the out projection of those "
-                       f"rows (scaled linearly to all rows); {spent:.1f} s of CPU work")}
+                       f"rows (scaled linearly to all rows)"
+                       + (f", after recomputing the {cfg.cache_len} context rows' k, v whole" if fresh else "")
+                       + f"; {spent:.1f} s of CPU work")}
 
 
 def stage_hbm(cfg, r, peaks):
@@ -709,7 +761,9 @@ def reference_arm(args):
     n_rows = 16
     if args.config.startswith("sublayer_"):
         wts = make_sublayer_weights(cfg.hidden, cfg.seed + 100)
-        sample = lambda i, seed: oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=seed)[1]
+        fresh = args.config.startswith("sublayer_fresh_")
+        sample = lambda i, seed: oracle_sublayer_sample(cfg, x, wts, n_rows, head=i % cfg.n_heads, seed=seed,
+                                                        fresh=fresh)[1]
         text = "each step: one head's share of an oracle sublayer step (see cpu_baseline of the ours arm)"
     else:
         sample = lambda i, seed: oracle_sample_step(cfg, x, n_rows, head=i % cfg.n_heads, seed=seed)[1]
@@ -726,7 +780,8 @@ def reference_arm(args):
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": describe(cfg)},
+            "config": {"workload": describe(cfg) + ("; context k, v recomputed before every step"
+                                                    if args.config.startswith("sublayer_fresh_") else "")},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -783,7 +838,7 @@ def main():
         if rank == 0:
             line = sublayer_line(args, world, cfg, r)
             if world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = sublayer_cpu_baseline(cfg)
+                line["cpu_baseline"] = sublayer_cpu_baseline(cfg, fresh=args.config.startswith("sublayer_fresh_"))
             print(json.dumps(line), flush=True)
         if world > 1:
             import torch.distributed as dist

@@ -18,6 +18,9 @@
  *   B   the DiT attention sublayer around A2 (pre-norm, q/k/v and output projections on
  *       caller-supplied weights): dp_ln_modulate, dp_linear, dp_qkv_project,
  *       dp_out_project, dp_sublayer_step
+ *   C   the fresh-context variant of the cache (context K/V recomputed at the step that
+ *       uses them, not reused from the block's last evaluation): dp_context_refresh,
+ *       dp_context_refresh_sublayer
  *
  * Conventions (all entry points):
  *  - Token tensors are row-major [rows][hidden], hidden = n_heads * head_dim, channel
@@ -331,6 +334,43 @@ dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, c
                            dp_kvcache* cache, void* work, void* out, int32_t n_heads,
                            int32_t head_dim, uint32_t flags, dp_queue* queue,
                            const void* push_noise, int64_t push_rows, void* stream);
+
+/* ---------------------------------------------------------------- fresh context (cache ablation) */
+
+/*
+ * The cached variant reuses the context block's K/V as its last evaluation produced them,
+ * one denoising step stale (the review's Section 3.2; the referee asks for an ablation
+ * against K/V recomputed at the current step).  These calls recompute them instead: the
+ * context rows go through the same feature projection as the window's own rows, with the
+ * conditioning the caller gives for the current step, and the result overwrites the cache
+ * slot the next step's attention reads (the most recently written slot; slot 0 before the
+ * first advance).  That slot's len becomes n_ctx; n_advances and the other slots are
+ * unchanged.  A following dp_window_step / dp_sublayer_step (same stream) attends to the
+ * recomputed rows; with DP_STEP_CACHE_ALL_SLOTS the older slots keep their cached rows.
+ * ctx_blk is the block table of the context rows (usually one block; mod[b] = that
+ * block's adaLN vectors at the timestep it is conditioned on now); ctx_blk->hidden is
+ * the hidden size.  n_ctx = 0 empties the slot and enqueues nothing.  CAPACITY if n_ctx
+ * exceeds the cache capacity.  The context rows and scratch overlap no slot of the cache
+ * ring (INVALID_ARG).
+ */
+
+/* Window-step features (identity projections, as in dp_window_step): k' = k_ctx (1 +
+ * scale_b) + shift_b and v' likewise, b = the context block of the row, one fp32 fma
+ * rounded once to the feature type.  k_ctx, v_ctx: DEVICE [n_ctx][hidden] of dt (DP_BF16
+ * with an f16 cache, or DP_F32 with an f32 cache); they may be the same rows. */
+dp_status dp_context_refresh(const void* k_ctx, const void* v_ctx, int64_t n_ctx, const dp_blocks* ctx_blk,
+                             dp_kvcache* cache, dp_dtype dt, void* stream);
+
+/* Sublayer features (as in dp_sublayer_step): h = LN(x_ctx) (1 + scale_b) + shift_b in bf16
+ * (B1, eps as in dp_ln_modulate), then k = h W_k^T + b_k and v = h W_v^T + b_v in f16
+ * (saturating), W_k and W_v rows [hidden, 2 hidden) and [2 hidden, 3 hidden) of w_qkv
+ * (DEVICE [3 hidden][hidden] bf16), b_k and b_v the same entries of b_qkv (DEVICE float or
+ * NULL).  x_ctx: DEVICE [n_ctx][hidden] bf16; work: DEVICE scratch of n_ctx * hidden bf16
+ * elements, overlapping neither x_ctx nor the cache; the cache holds f16 features; hidden
+ * a multiple of 256. */
+dp_status dp_context_refresh_sublayer(const void* x_ctx, int64_t n_ctx, const dp_blocks* ctx_blk,
+                                      const void* w_qkv, const float* b_qkv, float eps,
+                                      dp_kvcache* cache, void* work, void* stream);
 
 /* ---------------------------------------------------------------- profiling */
 

@@ -88,6 +88,9 @@ _SIGS = {
     "dp_out_project": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), _P, _P, _P],
     "dp_sublayer_step": [_P, _I64, ctypes.POINTER(DpBlocks), _P, _P, _P, _P, _F, ctypes.POINTER(DpKvcache), _P, _P,
                          _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _P],
+    "dp_context_refresh": [_P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _I32, _P],
+    "dp_context_refresh_sublayer": [_P, _I64, ctypes.POINTER(DpBlocks), _P, _P, _F, ctypes.POINTER(DpKvcache), _P,
+                                    _P],
     "dp_profile_begin": [_I32],
     "dp_profile_end": [ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_F), ctypes.POINTER(_I32)],
     "dp_profile_end_stages": [ctypes.POINTER(_F), _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I32)],
@@ -461,6 +464,30 @@ def sublayer_step(x, blocks: DpBlocks, w_qkv, b_qkv, w_o, b_o, cache: KVCache, w
                                  (STEP_POP if pop else 0) | (STEP_CACHE_ALL_SLOTS if cache_all_slots else 0),
                                  ctypes.byref(queue.desc) if queue is not None else None,
                                  _ptr(push_noise), int(rows), _stream(ref, stream)), "dp_sublayer_step")
+
+
+# ------------------------------------------------------------------------- C: fresh context
+
+def context_refresh(k_ctx, v_ctx, ctx_blocks: DpBlocks, cache: KVCache, stream=None) -> None:
+    """Recompute the context K/V of the window step now (dp_context_refresh): k' = k_ctx *
+    (1 + scale_b) + shift_b, v' likewise, written over the cache slot the next step reads;
+    k_ctx, v_ctx [n_ctx][hidden] bf16 (f16 cache) or f32 (f32 cache)."""
+    _check(_lib.dp_context_refresh(_ptr(k_ctx), _ptr(v_ctx), k_ctx.shape[0], ctypes.byref(ctx_blocks),
+                                   ctypes.byref(cache.desc), _dtype(k_ctx), _stream(k_ctx, stream)),
+           "dp_context_refresh")
+
+
+def context_refresh_sublayer(x_ctx, ctx_blocks: DpBlocks, w_qkv, b_qkv, cache: KVCache, work,
+                             eps: float = LN_EPS, stream=None) -> None:
+    """Recompute the context K/V of the sublayer now (dp_context_refresh_sublayer): pre-norm
+    with the context block's adaLN vectors, then the k and v thirds of the q/k/v projection,
+    written over the cache slot the next step reads; x_ctx [n_ctx][hidden] bf16, work at
+    least n_ctx * hidden bf16 elements (e.g. sublayer_work's first plane)."""
+    if work.numel() * work.element_size() < x_ctx.numel() * 2:
+        raise ValueError("work holds fewer than n_ctx * hidden 16-bit elements")
+    _check(_lib.dp_context_refresh_sublayer(_ptr(x_ctx), x_ctx.shape[0], ctypes.byref(ctx_blocks), _ptr(w_qkv),
+                                            _ptr(b_qkv), float(eps), ctypes.byref(cache.desc), _ptr(work),
+                                            _stream(x_ctx, stream)), "dp_context_refresh_sublayer")
 
 
 def sublayer_planes(work, n_win: int, hidden: int):

@@ -782,6 +782,101 @@ dp_status dp_out_project(const void* o, const void* w_o, const float* b_o, int64
   return run_out(o, w_o, b_o, n_rows, blk, residual, out, static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// Checks shared by the fresh-context entry points: the context fits the slot the next
+// attention reads, and the block table covers the context rows.  Returns that slot's k/v
+// row pointers.
+dp_status check_context(const dp_kvcache* cache, int64_t n_ctx, const dp_blocks* ctx_blk, dp_dtype feat,
+                        char** ck, char** cv) {
+  if (!ctx_blk) return fail(DP_ERR_INVALID_ARG, "context block table is NULL");
+  dp_status st = check_cache(cache, ctx_blk->hidden, feat);
+  if (st != DP_OK) return st;
+  if (n_ctx < 0 || n_ctx > INT32_MAX) return fail(DP_ERR_INVALID_ARG, "n_ctx %lld", static_cast<long long>(n_ctx));
+  if (n_ctx > cache->capacity)
+    return fail(DP_ERR_CAPACITY, "context of %lld rows > cache capacity %lld", static_cast<long long>(n_ctx),
+                static_cast<long long>(cache->capacity));
+  st = check_blocks(ctx_blk, n_ctx, ctx_blk->hidden);
+  if (st != DP_OK) return st;
+  const int64_t slot_bytes = cache->capacity * ctx_blk->hidden * elem_bytes(feat);
+  const int64_t slot = cache_read_slot(cache);
+  *ck = static_cast<char*>(cache->k) + slot * slot_bytes;
+  *cv = static_cast<char*>(cache->v) + slot * slot_bytes;
+  return DP_OK;
+}
+
+// True when [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + static_cast<uintptr_t>(nb) && y < x + static_cast<uintptr_t>(na);
+}
+
+}  // namespace
+
+dp_status dp_context_refresh(const void* k_ctx, const void* v_ctx, int64_t n_ctx, const dp_blocks* ctx_blk,
+                             dp_kvcache* cache, dp_dtype dt, void* stream) {
+  if (dt != DP_BF16 && dt != DP_F32) return fail(DP_ERR_UNSUPPORTED, "context dtype %d (bf16 or f32)", dt);
+  const dp_dtype feat = feature_dtype(dt);
+  char* ck = nullptr;
+  char* cv = nullptr;
+  dp_status st = check_context(cache, n_ctx, ctx_blk, feat, &ck, &cv);
+  if (st != DP_OK) return st;
+  const int32_t hidden = ctx_blk->hidden;
+  if (!hidden_ok(hidden, dt)) return fail(DP_ERR_INVALID_ARG, "hidden %d not a whole number of 16-byte vectors", hidden);
+  if (!k_ctx || !v_ctx || !aligned16(k_ctx) || !aligned16(v_ctx))
+    return fail(DP_ERR_INVALID_ARG, "k_ctx/v_ctx NULL or misaligned");
+  const int64_t in_bytes = n_ctx * hidden * elem_bytes(dt);
+  const int64_t ring_bytes = cache->n_slots * cache->capacity * hidden * elem_bytes(feat);
+  if (overlaps(k_ctx, in_bytes, cache->k, ring_bytes) || overlaps(k_ctx, in_bytes, cache->v, ring_bytes) ||
+      overlaps(v_ctx, in_bytes, cache->k, ring_bytes) || overlaps(v_ctx, in_bytes, cache->v, ring_bytes))
+    return fail(DP_ERR_INVALID_ARG, "context rows overlap the cache ring");
+  if (n_ctx > 0) {
+    const void* src[2] = {k_ctx, v_ctx};
+    void* dst[2] = {ck, cv};
+    cudaError_t e = dp::launch_modulate(src, dst, 2, n_ctx, hidden, to_table(ctx_blk), dt, feat,
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "context modulate launch");
+  }
+  cache->len[cache_read_slot(cache)] = n_ctx;
+  return DP_OK;
+}
+
+dp_status dp_context_refresh_sublayer(const void* x_ctx, int64_t n_ctx, const dp_blocks* ctx_blk, const void* w_qkv,
+                                      const float* b_qkv, float eps, dp_kvcache* cache, void* work, void* stream) {
+  char* ck = nullptr;
+  char* cv = nullptr;
+  dp_status st = check_context(cache, n_ctx, ctx_blk, DP_F16, &ck, &cv);
+  if (st != DP_OK) return st;
+  const int32_t hidden = ctx_blk->hidden;
+  if (n_ctx > 0) {
+    st = check_ln(x_ctx, work, n_ctx, ctx_blk, eps);
+    if (st != DP_OK) return st;
+    st = check_linear(work, w_qkv, b_qkv, n_ctx, 3 * static_cast<int64_t>(hidden), hidden);
+    if (st != DP_OK) return st;
+    const int64_t plane = n_ctx * hidden * 2;
+    const int64_t ring_bytes = cache->n_slots * cache->capacity * hidden * 2;
+    if (overlaps(work, plane, x_ctx, plane) || overlaps(work, plane, cache->k, ring_bytes) ||
+        overlaps(work, plane, cache->v, ring_bytes) || overlaps(x_ctx, plane, cache->k, ring_bytes) ||
+        overlaps(x_ctx, plane, cache->v, ring_bytes))
+      return fail(DP_ERR_INVALID_ARG, "x_ctx, work and the cache ring must not overlap");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // B1 on the context rows, then the k and v thirds of the q/k/v projection
+    st = run_ln(x_ctx, work, n_ctx, ctx_blk, eps, s);
+    if (st != DP_OK) return st;
+    const int64_t w_off = static_cast<int64_t>(hidden) * hidden * 2;
+    dp::GemmArgs g = gemm_args(work, static_cast<const char*>(w_qkv) + w_off, b_qkv ? b_qkv + hidden : nullptr,
+                               n_ctx, 2 * hidden, hidden, dp::kEpiKV);
+    g.y1 = ck;
+    g.y2 = cv;
+    g.ld_y = hidden;
+    g.seg_cols = hidden;
+    st = run_gemm(g, s, "context k/v projection launch");
+    if (st != DP_OK) return st;
+  }
+  cache->len[cache_read_slot(cache)] = n_ctx;
+  return DP_OK;
+}
+
 dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, const void* w_qkv, const float* b_qkv,
                            const void* w_o, const float* b_o, float eps, dp_kvcache* cache, void* work, void* out,
                            int32_t n_heads, int32_t head_dim, uint32_t flags, dp_queue* queue,

@@ -82,10 +82,10 @@ struct GemmParams {
   int32_t n_tiles;
   const float* bias;               // [n] or NULL
   void* y0;                        // kEpiStore: y; kEpiQKV: q; kEpiGateResidual: y
-  void* y1;                        // kEpiQKV: k
-  void* y2;                        // kEpiQKV: v
+  void* y1;                        // kEpiQKV, kEpiKV: k
+  void* y2;                        // kEpiQKV, kEpiKV: v
   int32_t ld_y;                    // row pitch of the outputs, elements
-  int32_t seg_cols;                // kEpiQKV: columns per q/k/v segment (hidden)
+  int32_t seg_cols;                // kEpiQKV, kEpiKV: columns per q/k/v segment (hidden)
   int32_t y_f16;                   // kEpiStore: output f16 (1) or bf16 (0)
   const __nv_bfloat16* residual;   // kEpiGateResidual: [m][n]
   uint32_t* status;
@@ -113,10 +113,12 @@ __device__ __forceinline__ void store32(const GemmParams& p, int64_t row, int co
                        : make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                                     pack_bf16x2(f[6], f[7]));
     }
-  } else if constexpr (EPI == kEpiQKV) {
-    // q (bf16, the attention's raw query) | k | v (f16 features, saturating)
-    const int seg = col / p.seg_cols;
-    const int cin = col - seg * p.seg_cols;
+  } else if constexpr (EPI == kEpiQKV || EPI == kEpiKV) {
+    // q (bf16, the attention's raw query) | k | v (f16 features, saturating); kEpiKV has
+    // no q columns
+    const int sc = col / p.seg_cols;
+    const int cin = col - sc * p.seg_cols;
+    const int seg = (EPI == kEpiKV ? 1 : 0) + sc;
     void* base = seg == 0 ? p.y0 : (seg == 1 ? p.y1 : p.y2);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(base) + row * p.ld_y + cin);
 #pragma unroll
@@ -371,7 +373,7 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
 template <int EPI>
 cudaError_t launch_epi(const GemmArgs& g, cudaStream_t s) {
   // the widest tile that divides the columns (and, for q/k/v, each segment)
-  const int32_t unit = EPI == kEpiQKV ? g.seg_cols : g.n;
+  const int32_t unit = (EPI == kEpiQKV || EPI == kEpiKV) ? g.seg_cols : g.n;
   if (unit % 256 == 0) return launch_bn<256, EPI>(g, s);
   return launch_bn<128, EPI>(g, s);
 }
@@ -384,6 +386,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     case kEpiStore: return launch_epi<kEpiStore>(g, s);
     case kEpiQKV: return launch_epi<kEpiQKV>(g, s);
     case kEpiGateResidual: return launch_epi<kEpiGateResidual>(g, s);
+    case kEpiKV: return launch_epi<kEpiKV>(g, s);
     default: return cudaErrorInvalidValue;
   }
 }

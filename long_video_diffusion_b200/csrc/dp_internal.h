@@ -109,6 +109,7 @@ enum GemmEpi {
   kEpiStore = 0,         // y0 [m][ld_y], bf16 or f16 (y_f16)
   kEpiQKV = 1,           // columns [0, s) -> y0 (q, bf16), [s, 2s) -> y1 (k, f16), [2s, 3s) -> y2 (v, f16)
   kEpiGateResidual = 2,  // y0 = residual + gate_b * (a W^T + bias), bf16; b = block of the row
+  kEpiKV = 3,            // columns [0, s) -> y1 (k, f16), [s, 2s) -> y2 (v, f16)
 };
 
 struct GemmArgs {

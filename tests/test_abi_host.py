@@ -249,3 +249,31 @@ def test_sublayer_entry_points_check_before_launch(m):
     assert c.n_advances == 0
     assert step(out=FAKE) == m.ERR_INVALID_ARG                  # out aliases x
     assert step(hd=32) == m.ERR_UNSUPPORTED                     # attention head_dim
+
+
+def test_context_refresh_checks_before_launch(m):
+    P = ctypes.c_void_p
+    c = _cache(m, capacity=128, hidden=128, length=77)
+    ref = lambda n=100, k=FAKE, v=FAKE + 65536, dt=1, rows=None, cache=c: m._lib.dp_context_refresh(
+        P(k), P(v), n, ctypes.byref(_blocks(m, [n] if rows is None else rows, 128)), ctypes.byref(cache), dt, None)
+    assert ref(dt=2) == m.ERR_UNSUPPORTED                        # f16 context rows
+    assert ref(dt=0) == m.ERR_INVALID_ARG                        # f32 rows need an f32 cache
+    assert ref(n=129) == m.ERR_CAPACITY                          # more rows than the slot holds
+    assert ref(k=0) == m.ERR_INVALID_ARG
+    assert ref(v=FAKE + 8) == m.ERR_INVALID_ARG                  # misaligned
+    assert ref(k=FAKE + (1 << 20)) == m.ERR_INVALID_ARG          # rows inside the cache ring
+    assert ref(rows=[50, 49]) == m.ERR_INVALID_ARG               # block table covers 99 of 100 rows
+    assert c.len[0] == 77
+    assert ref(n=0) == m.OK and c.len[0] == 0                    # empty context: nothing enqueued
+    c2 = _cache(m, capacity=128, hidden=256, length=5)
+    sub = lambda n=100, x=FAKE, work=FAKE + (4 << 20), eps=1e-6, hidden=256, cache=c2: \
+        m._lib.dp_context_refresh_sublayer(P(x), n, ctypes.byref(_blocks(m, [n], hidden)), P(FAKE + (8 << 20)),
+                                           None, eps, ctypes.byref(cache), P(work), None)
+    assert sub(n=200) == m.ERR_CAPACITY
+    assert sub(eps=0.0) == m.ERR_INVALID_ARG
+    assert sub(hidden=128, cache=_cache(m, capacity=128, hidden=128)) == m.ERR_UNSUPPORTED
+    assert sub(work=FAKE + 4096) == m.ERR_INVALID_ARG            # work overlaps x_ctx
+    assert sub(work=FAKE + (2 << 20)) == m.ERR_INVALID_ARG       # work overlaps the cache ring
+    assert sub(x=0) == m.ERR_INVALID_ARG
+    assert c2.len[0] == 5
+    assert sub(n=0) == m.OK and c2.len[0] == 0
