@@ -238,7 +238,9 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     (all 850 by default) of a fresh run are timed.  long_run_ctx4: the cache holds the last
     four exited blocks (8 latent frames, the pages' NumC = 8) and every step attends to all
     of them.  long_run_coord: blocks are pushed with the coordinated noise initialisation
-    (frames of a pool holding the first window's noise, in a fresh random order per block)."""
+    (frames of a pool holding the first window's noise, in a fresh random order per block).
+    long_run_fresh: before every step the context K/V are recomputed from the exited block's
+    latent rows (conditioned on timestep 0, where its last evaluation ran) instead of reused."""
     import torch
     import torch.distributed as dist
 
@@ -259,6 +261,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     stream = torch.cuda.current_stream(dev)
 
     n_ctx = 4 if args.config == "long_run_ctx4" else 1
+    fresh_t = 0 if args.config == "long_run_fresh" else None
     frame_pool = None
     if args.config == "long_run_coord":
         pool = make_run_pool(rc).to(dev)
@@ -269,23 +272,23 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
             lists.append(dp.coordinated_frames(pool.shape[0], nf[b], lists[b - 1], perms[b]))
         frame_pool = (pool, lists)
 
-    def fresh():
+    def new_state():
         return (dp.KVCache(rc.slot_rows, D, torch.float16, n_slots=n_ctx, device=dev),
-                dp.Queue(W, rc.slot_rows, D, device=dev))
+                dp.Queue(W + (1 if fresh_t is not None else 0), rc.slot_rows, D, device=dev))
 
     def cache_rows_read(c):
         return sum(c.desc.len[i] for i in range(n_ctx)) if n_ctx > 1 else c.length
 
-    cache, queue = fresh()
+    cache, queue = new_state()
     dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, max_steps=args.warmup,
-                cache_all_slots=n_ctx > 1, frame_pool=frame_pool)
+                cache_all_slots=n_ctx > 1, frame_pool=frame_pool, fresh_t=fresh_t)
     torch.cuda.synchronize()
     dp.device_status()
 
     # per-step attention work: 4 n (L_c + n) hd H with L_c the cache length before the step
     steps_n, steps_lc = [], []
-    cache, queue = fresh()
-    state = {"lc": 0}
+    cache, queue = new_state()
+    state = {"lc": 0, "exited": False}
 
     launches = [0]
 
@@ -293,6 +296,9 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         steps_n.append(n)
         steps_lc.append(state["lc"])
         state["lc"] = cache_rows_read(cache)
+        if fresh_t is not None and state["exited"]:
+            launches[0] += 1     # the context recompute before the step
+        state["exited"] = state["exited"] or popped
         if frame_pool is None:   # modulate, attention (+ one copy for the pop and the push)
             launches[0] += 2 + (1 if (popped or pushed is not None) else 0)
         else:                    # modulate, attention (+ the pop's copy) (+ the push's gather)
@@ -309,7 +315,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     dp.profile_begin(args.steps)
     t0.record(stream)
     n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps,
-                          cache_all_slots=n_ctx > 1, frame_pool=frame_pool)
+                          cache_all_slots=n_ctx > 1, frame_pool=frame_pool, fresh_t=fresh_t)
     t1.record(stream)
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
@@ -344,7 +350,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         hout[:n].copy_(out[:n], non_blocking=True)
         d2h[0] += n * D * 2
 
-    cache, queue = fresh()
+    cache, queue = new_state()
     e2e_pool = None
     if frame_pool is not None:   # the pool is the run's input: copied from pinned host memory once
         hpool = frame_pool[0].cpu().pin_memory()
@@ -359,7 +365,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     if e2e_pool is not None:
         e2e_pool[0].copy_(hpool, non_blocking=True)
     n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps,
-                        cache_all_slots=n_ctx > 1, frame_pool=e2e_pool)
+                        cache_all_slots=n_ctx > 1, frame_pool=e2e_pool, fresh_t=fresh_t)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -369,7 +375,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     ms, e2e_ms, attn_ms = max_over_ranks([ms, e2e_ms, attn_ms], dev)
     return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
                 e2e_ms=e2e_ms, e2e_steps=n_e2e, h2d=hb.h2d / max(n_e2e, 1), d2h=d2h[0] / max(n_e2e, 1),
-                clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx)
+                clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx, fresh=fresh_t is not None)
 
 
 def long_run_line(args, world, r):
@@ -385,13 +391,16 @@ def long_run_line(args, world, r):
         "config": {"workload": (f"{args.config}: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
                                 f"{rc.frames_per_block}-frame blocks, window of {rc.window_blocks} blocks, "
                                 f"{rc.n_timesteps} staggered timesteps per block, {rc.n_heads}x{rc.head_dim} heads, "
-                                f"bf16, cache of the last {r['n_ctx']} exited block(s); first {r['steps']} schedule steps"),
+                                f"bf16, cache of the last {r['n_ctx']} exited block(s)"
+                                + ("; context K/V recomputed before every step (timestep 0)" if r["fresh"] else "")
+                                + f"; first {r['steps']} schedule steps"),
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "steady-state window q = k = v 66 MiB plus k', v', cache and out: 265 MiB per step > 126 MiB"},
         "window_tokens": r["tokens"],
         "attn_tflops": achieved,
         "stage_ms": {"modulate": r["mod_ms"] / r["steps"], "attention": r["attn_ms"] / r["steps"],
-                     "advance": r["adv_ms"] / r["steps"]},
+                     "advance": r["adv_ms"] / r["steps"],
+                     "outside_stages": (r["ms"] - r["mod_ms"] - r["attn_ms"] - r["adv_ms"]) / r["steps"]},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
                      "traffic_unit": "bytes per launch (not captured for the run: window sizes vary per step)",
@@ -817,7 +826,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    if args.config in ("long_run", "long_run_ctx4", "long_run_coord"):
+    if args.config in ("long_run", "long_run_ctx4", "long_run_coord", "long_run_fresh"):
         if args.steps == 300 and "--steps" not in sys.argv:
             args.steps = 850                 # the whole run
         r = long_run_arm(args, rank, world, local_rank)

@@ -572,7 +572,7 @@ def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
              queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
              on_step=None, stream=None, max_steps: Optional[int] = None, cache_all_slots: bool = False,
-             frame_pool=None) -> int:
+             frame_pool=None, fresh_t: Optional[int] = None) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
@@ -581,9 +581,16 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
     are then left mid-run).  cache_all_slots: every step attends to all of the cache ring's
     slots (the last n_slots exited blocks).  frame_pool = (pool, frame_lists): blocks are
     pushed as pool frames (dp_queue_push_frames; the coordinated noise initialisation) and
-    noise_blocks only gives each block's row count.  Returns the number of steps."""
+    noise_blocks only gives each block's row count.  fresh_t: before every step after the
+    first exit, the context K/V are recomputed (dp_context_refresh) from the latent rows of
+    the block that left last, conditioned on table[fresh_t], instead of reused from its last
+    evaluation; the queue keeps those rows in the slot behind its head, so it needs more
+    slots than window_blocks.  Returns the number of steps."""
     T = len(tau)
     n_blocks = len(noise_blocks)
+    if fresh_t is not None and queue.desc.n_slots <= window_blocks:
+        raise ValueError("a fresh context needs a queue with more slots than window blocks")
+    exited_rows = 0
     def push_block(b):
         if frame_pool is None:
             queue_push(queue, noise_blocks[b], stream=stream)
@@ -594,8 +601,13 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
     nxt = 1
     step = 0
     while queue.count > 0 and (max_steps is None or step < max_steps):
+        if fresh_t is not None and exited_rows > 0:
+            ctx = queue.latent[(queue.head - 1) % queue.desc.n_slots, :exited_rows]
+            context_refresh(ctx, ctx, blocks_from_table(table, [fresh_t], [exited_rows]), cache, stream=stream)
         blk, win, n = queue_blocks(queue, table, tau)
         pop = queue.evals()[0] + 1 == T
+        if pop:
+            exited_rows = queue.rows()[0]
         push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1
         fused_push = push and frame_pool is None
         window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,

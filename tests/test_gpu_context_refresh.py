@@ -190,3 +190,50 @@ def test_refresh_writes_only_the_slot_attention_reads(dp):
     mod = O.lookup(table, [0, 999])
     want, _, _ = O.window_step(q.cpu(), k.cpu(), v.cpu(), ck, cv, ck.shape[0], [0, 128, n], mod, H, hd)
     assert_close(out_all.cpu().double().numpy(), want, "bf16", "every slot, slot 0 refreshed")
+
+
+# ----------------------------------------------------------------------------- the long run
+
+def _long_run_sums(dp, fresh_t, max_steps=None):
+    """Per-step checksums of the long run's outputs (int64 sums of the bf16 bit patterns)."""
+    from workloads import make_run_noise, make_run_table, run_config
+    rc = run_config()
+    H, hd, D, W, T = rc.n_heads, rc.head_dim, rc.hidden, rc.window_blocks, rc.n_timesteps
+    noise = [b.cuda() for b in make_run_noise(rc)]
+    table = make_run_table(rc).cuda()
+    tau = O.timestep_schedule(T)
+    cache = dp.KVCache(rc.slot_rows, D, torch.float16)
+    queue = dp.Queue(W + 1, rc.slot_rows, D)
+    n_max = W * rc.slot_rows
+    kv = torch.empty(2 * n_max * D, dtype=torch.float16, device="cuda")
+    out = torch.empty(n_max, D, dtype=torch.bfloat16, device="cuda")
+    sums, pops = [], []
+
+    def on_step(step, n, popped, pushed):
+        sums.append(out[:n].view(torch.int16).sum(dtype=torch.int64))
+        pops.append(popped)
+
+    steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=max_steps,
+                        fresh_t=fresh_t)
+    dp.device_status()
+    return torch.stack(sums).cpu(), pops, steps
+
+
+def test_long_run_fresh_context_at_the_final_timestep_equals_cached(dp):
+    """The whole run with the context recomputed before every step from the exited block's
+    latent rows at timestep 0 (where its last evaluation ran) gives the cached run's outputs
+    bit for bit at every one of the 850 steps; conditioned on another timestep it does not."""
+    cached, pops, n = _long_run_sums(dp, None)
+    fresh, pops_f, n_f = _long_run_sums(dp, 0)
+    assert n == n_f == 850 and pops == pops_f
+    assert torch.equal(cached, fresh)
+    first_exit = pops.index(True)
+    other, _, _ = _long_run_sums(dp, 500, max_steps=first_exit + 3)
+    assert torch.equal(other[:first_exit + 1], cached[:first_exit + 1])   # no context yet, or the same one
+    assert not torch.equal(other[first_exit + 1:], cached[first_exit + 1:first_exit + 3])
+    with pytest.raises(ValueError):
+        from workloads import run_config
+        rc = run_config()
+        q = dp.Queue(rc.window_blocks, rc.slot_rows, rc.hidden)
+        dp.run_fifo([], torch.zeros(1000, 3, rc.hidden, device="cuda"), [0], rc.window_blocks,
+                    dp.KVCache(rc.slot_rows, rc.hidden, torch.float16), q, None, None, 1, 1, fresh_t=0)
