@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -717,9 +718,9 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool attr_set[64] = {};  // per instantiation and device
+  static std::atomic<bool> attr_set[64];  // per instantiation and device (concurrent first calls both set it)
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(window_attn_tc_kernel<HD, F16, MULTI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              L::ALLOC);
     if (e != cudaSuccess) return e;
@@ -729,7 +730,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
     e = cudaFuncGetAttributes(&fa, window_attn_tc_kernel<HD, F16, MULTI>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < L::kLaunchRegs) return cudaErrorInvalidConfiguration;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t grid = static_cast<int64_t>(p.n_qpairs) * a.n_heads;
   window_attn_tc_kernel<HD, F16, MULTI><<<static_cast<unsigned>(grid), L::kThreads, L::ALLOC, s>>>(tkc, tvc, tkw, tvw,

@@ -28,6 +28,7 @@
 // blocks of W (about 27 MB at hidden 3072) instead of whole rows of W.
 // Every wait is bounded (dp_device.cuh): on giving up the kernel records a timeout in the
 // device status word, stops, drains its own copies and products, frees TMEM and returns.
+#include <atomic>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -355,12 +356,12 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool attr_set[64] = {};  // per instantiation and device
+  static std::atomic<bool> attr_set[64];  // per instantiation and device (concurrent first calls both set it)
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   int sms = 148;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
