@@ -189,6 +189,19 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
     clocks = sampler.stop() if sampler else None
+    # per-step times of the full-window (steady-state) steps, early and late in the run: the
+    # step's work depends on the block size, not on how much video came before
+    step_ms = [(step_ev[i - 1] if i else t0).elapsed_time(step_ev[i]) for i in range(len(step_ev))]
+    full = [i for i, nn in enumerate(steps_n) if nn == max(steps_n)]
+    steady = {}
+    if len(full) >= 6:
+        third = len(full) // 3
+        pick = lambda idx: sorted(step_ms[i] for i in idx)
+        allv = pick(full)
+        steady = {"steps": len(full), "median_ms": statistics.median(allv),
+                  "p05_ms": allv[len(allv) // 20], "p95_ms": allv[(19 * len(allv)) // 20],
+                  "first_third_median_ms": statistics.median(pick(full[:third])),
+                  "last_third_median_ms": statistics.median(pick(full[-third:]))}
     if world > 1:
         dist.barrier()
     dp.device_status()
@@ -292,7 +305,12 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
 
     launches = [0]
 
+    step_ev = []
+
     def on_step(step, n, popped, pushed):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        step_ev.append(ev)
         steps_n.append(n)
         steps_lc.append(state["lc"])
         state["lc"] = cache_rows_read(cache)
@@ -320,6 +338,19 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
     clocks = sampler.stop() if sampler else None
+    # per-step times of the full-window (steady-state) steps, early and late in the run: the
+    # step's work depends on the block size, not on how much video came before
+    step_ms = [(step_ev[i - 1] if i else t0).elapsed_time(step_ev[i]) for i in range(len(step_ev))]
+    full = [i for i, nn in enumerate(steps_n) if nn == max(steps_n)]
+    steady = {}
+    if len(full) >= 6:
+        third = len(full) // 3
+        pick = lambda idx: sorted(step_ms[i] for i in idx)
+        allv = pick(full)
+        steady = {"steps": len(full), "median_ms": statistics.median(allv),
+                  "p05_ms": allv[len(allv) // 20], "p95_ms": allv[(19 * len(allv)) // 20],
+                  "first_third_median_ms": statistics.median(pick(full[:third])),
+                  "last_third_median_ms": statistics.median(pick(full[-third:]))}
     if world > 1:
         dist.barrier()
     dp.device_status()
@@ -375,7 +406,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     ms, e2e_ms, attn_ms = max_over_ranks([ms, e2e_ms, attn_ms], dev)
     return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
                 e2e_ms=e2e_ms, e2e_steps=n_e2e, h2d=hb.h2d / max(n_e2e, 1), d2h=d2h[0] / max(n_e2e, 1),
-                clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx, fresh=fresh_t is not None)
+                clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx, fresh=fresh_t is not None, steady=steady)
 
 
 def long_run_line(args, world, r):
@@ -397,6 +428,7 @@ def long_run_line(args, world, r):
                    "parallelism": f"replicas x{world} (no exchange)",
                    "l2": "steady-state window q = k = v 66 MiB plus k', v', cache and out: 265 MiB per step > 126 MiB"},
         "window_tokens": r["tokens"],
+        "full_window_step_ms": r["steady"],
         "attn_tflops": achieved,
         "stage_ms": {"modulate": r["mod_ms"] / r["steps"], "attention": r["attn_ms"] / r["steps"],
                      "advance": r["adv_ms"] / r["steps"],

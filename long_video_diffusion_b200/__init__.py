@@ -572,7 +572,7 @@ def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
              queue: Queue, kv_work: torch.Tensor, out: torch.Tensor, n_heads: int, head_dim: int,
              on_step=None, stream=None, max_steps: Optional[int] = None, cache_all_slots: bool = False,
-             frame_pool=None, fresh_t: Optional[int] = None) -> int:
+             frame_pool=None, fresh_t: Optional[int] = None, state: Optional["FifoState"] = None) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
@@ -585,30 +585,34 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
     first exit, the context K/V are recomputed (dp_context_refresh) from the latent rows of
     the block that left last, conditioned on table[fresh_t], instead of reused from its last
     evaluation; the queue keeps those rows in the slot behind its head, so it needs more
-    slots than window_blocks.  Returns the number of steps."""
+    slots than window_blocks.  state: the run's progress (FifoState), updated as steps are
+    enqueued; a run stopped by max_steps continues from it, also after checkpoint/restore.
+    Returns the number of steps run so far (state.step)."""
     T = len(tau)
     n_blocks = len(noise_blocks)
     if fresh_t is not None and queue.desc.n_slots <= window_blocks:
         raise ValueError("a fresh context needs a queue with more slots than window blocks")
-    exited_rows = 0
+    st = state if state is not None else FifoState()
     def push_block(b):
         if frame_pool is None:
             queue_push(queue, noise_blocks[b], stream=stream)
         else:
             queue_push_frames(queue, frame_pool[0], frame_pool[1][b], stream=stream)
 
-    push_block(0)
-    nxt = 1
-    step = 0
-    while queue.count > 0 and (max_steps is None or step < max_steps):
-        if fresh_t is not None and exited_rows > 0:
-            ctx = queue.latent[(queue.head - 1) % queue.desc.n_slots, :exited_rows]
-            context_refresh(ctx, ctx, blocks_from_table(table, [fresh_t], [exited_rows]), cache, stream=stream)
+    if st.nxt == 0:
+        push_block(0)
+        st.nxt = 1
+    run = 0
+    while queue.count > 0 and (max_steps is None or run < max_steps):
+        if fresh_t is not None and st.exited_rows > 0:
+            ctx = queue.latent[(queue.head - 1) % queue.desc.n_slots, :st.exited_rows]
+            context_refresh(ctx, ctx, blocks_from_table(table, [fresh_t], [st.exited_rows]), cache, stream=stream)
         blk, win, n = queue_blocks(queue, table, tau)
         pop = queue.evals()[0] + 1 == T
         if pop:
-            exited_rows = queue.rows()[0]
-        push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == step + 1
+            st.exited_rows = queue.rows()[0]
+        nxt = st.nxt
+        push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == st.step + 1
         fused_push = push and frame_pool is None
         window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,
                     push_noise=noise_blocks[nxt] if fused_push else None, stream=stream, n_win=n,
@@ -616,8 +620,60 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
         if push and not fused_push:
             push_block(nxt)
         if on_step is not None:
-            on_step(step, n, pop, nxt if push else None)
+            on_step(st.step, n, pop, nxt if push else None)
         if push:
-            nxt += 1
-        step += 1
-    return step
+            st.nxt += 1
+        st.step += 1
+        run += 1
+    return st.step
+
+
+class FifoState:
+    """Progress of a run_fifo run: steps taken, the next block to push (0 = none pushed yet)
+    and the row count of the block that left last."""
+
+    def __init__(self, step: int = 0, nxt: int = 0, exited_rows: int = 0):
+        self.step, self.nxt, self.exited_rows = step, nxt, exited_rows
+
+
+_QUEUE_FIELDS = ("slot_rows", "hidden", "n_slots", "head", "count", "n_pushed", "n_popped", "dtype")
+_CACHE_FIELDS = ("capacity", "hidden", "n_slots", "n_advances", "dtype")
+
+
+def checkpoint(queue: Queue, cache: KVCache, state: Optional[FifoState] = None) -> dict:
+    """Host copy of a run's state: the queue's and the cache's descriptors and device buffers
+    (copied to host memory after the work enqueued on the current stream), and the run's
+    progress.  The dict holds plain values and CPU tensors (torch.save-able)."""
+    qd, cd = queue.desc, cache.desc
+    return {
+        "queue": {**{f: getattr(qd, f) for f in _QUEUE_FIELDS},
+                  "rows": list(qd.rows), "evals": list(qd.evals)},
+        "queue_latent": queue.latent.cpu(),
+        "cache": {**{f: getattr(cd, f) for f in _CACHE_FIELDS}, "len": list(cd.len)},
+        "cache_k": cache.k.cpu(),
+        "cache_v": cache.v.cpu(),
+        "state": None if state is None else {"step": state.step, "nxt": state.nxt, "exited_rows": state.exited_rows},
+    }
+
+
+def restore(ckpt: dict, device="cuda"):
+    """(queue, cache, state) rebuilt from checkpoint(): new device buffers holding the saved
+    bytes, descriptors with the saved fields."""
+    q, c = ckpt["queue"], ckpt["cache"]
+    lat = ckpt["queue_latent"]
+    queue = Queue(q["n_slots"], q["slot_rows"], q["hidden"], dtype=lat.dtype, device=device)
+    queue.latent.copy_(lat)
+    for f in _QUEUE_FIELDS:
+        setattr(queue.desc, f, q[f])
+    for i in range(MAX_SLOTS):
+        queue.desc.rows[i], queue.desc.evals[i] = q["rows"][i], q["evals"][i]
+    k, v = ckpt["cache_k"], ckpt["cache_v"]
+    cache = KVCache(c["capacity"], c["hidden"], dtype=k.dtype, n_slots=c["n_slots"], device=device)
+    cache.k.copy_(k)
+    cache.v.copy_(v)
+    for f in _CACHE_FIELDS:
+        setattr(cache.desc, f, c[f])
+    for i in range(MAX_SLOTS):
+        cache.desc.len[i] = c["len"][i]
+    st = ckpt["state"]
+    return queue, cache, None if st is None else FifoState(**st)

@@ -83,3 +83,44 @@ def test_long_run_matches_oracle(dp):
     for step, (got, rows) in sorted(results.items()):
         want, ro, t, L = run.step(step, rows=rows)
         assert_close(got, want, "bf16", f"long run step {step}")
+
+
+def test_long_run_checkpoint_and_resume_is_bit_identical(dp):
+    """The run stopped at a steady-state step, checkpointed to host memory through
+    torch.save, restored into new buffers and continued gives, at every later step, the
+    outputs of the uninterrupted run bit for bit, and the same final cache and queue."""
+    import io
+    rc = run_config()
+    H, hd, D, W, T = rc.n_heads, rc.head_dim, rc.hidden, rc.window_blocks, rc.n_timesteps
+    noise = [b.cuda() for b in make_run_noise(rc)]
+    table = make_run_table(rc).cuda()
+    tau = O.timestep_schedule(T)
+    n_max = W * rc.slot_rows
+    kv = torch.empty(2 * n_max * D, dtype=torch.float16, device="cuda")
+    out = torch.empty(n_max, D, dtype=torch.bfloat16, device="cuda")
+
+    def sums_into(lst):
+        return lambda step, n, popped, pushed: lst.append(out[:n].view(torch.int16).sum(dtype=torch.int64))
+
+    ref = []
+    cache, queue = dp.KVCache(rc.slot_rows, D, torch.float16), dp.Queue(W, rc.slot_rows, D)
+    assert dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=sums_into(ref)) == 850
+    got = []
+    cache2, queue2 = dp.KVCache(rc.slot_rows, D, torch.float16), dp.Queue(W, rc.slot_rows, D)
+    state = dp.FifoState()
+    assert dp.run_fifo(noise, table, tau, W, cache2, queue2, kv, out, H, hd, on_step=sums_into(got),
+                       max_steps=300, state=state) == 300
+    buf = io.BytesIO()
+    torch.save(dp.checkpoint(queue2, cache2, state), buf)
+    del queue2, cache2
+    kv.fill_(0)
+    buf.seek(0)
+    queue3, cache3, state3 = dp.restore(torch.load(buf))
+    assert state3.step == 300
+    assert dp.run_fifo(noise, table, tau, W, cache3, queue3, kv, out, H, hd, on_step=sums_into(got),
+                       state=state3) == 850
+    dp.device_status()
+    assert torch.equal(torch.stack(got).cpu(), torch.stack(ref).cpu())
+    assert cache3.desc.n_advances == cache.desc.n_advances == len(noise) and cache3.length == cache.length
+    assert bytes_equal(cache3.k, cache.k) and bytes_equal(cache3.v, cache.v)
+    assert queue3.count == queue.count == 0 and queue3.desc.n_popped == queue.desc.n_popped
