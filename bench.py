@@ -189,19 +189,6 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     mod_ms, attn_ms, adv_ms, n_prof = dp.profile_end()
     clocks = sampler.stop() if sampler else None
-    # per-step times of the full-window (steady-state) steps, early and late in the run: the
-    # step's work depends on the block size, not on how much video came before
-    step_ms = [(step_ev[i - 1] if i else t0).elapsed_time(step_ev[i]) for i in range(len(step_ev))]
-    full = [i for i, nn in enumerate(steps_n) if nn == max(steps_n)]
-    steady = {}
-    if len(full) >= 6:
-        third = len(full) // 3
-        pick = lambda idx: sorted(step_ms[i] for i in idx)
-        allv = pick(full)
-        steady = {"steps": len(full), "median_ms": statistics.median(allv),
-                  "p05_ms": allv[len(allv) // 20], "p95_ms": allv[(19 * len(allv)) // 20],
-                  "first_third_median_ms": statistics.median(pick(full[:third])),
-                  "last_third_median_ms": statistics.median(pick(full[-third:]))}
     if world > 1:
         dist.barrier()
     dp.device_status()
