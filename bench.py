@@ -361,11 +361,27 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
             return self.dev[:h.shape[0]]
 
     hb = _HostBlocks(noise_cpu)
-    hout = torch.empty(n_max, D, dtype=torch.bfloat16).pin_memory()
+    # each step's output is read back on a copy stream while the next step computes: the
+    # steps alternate between two output buffers, and a step waits for the readback of the
+    # buffer it is about to overwrite
+    outs = [out, torch.empty_like(out)]
+    houts = [torch.empty(n_max, D, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    d2h_stream = torch.cuda.Stream(dev)
+    read_done = [None, None]
     d2h = [0]
 
     def on_step_e2e(step, n, popped, pushed):
-        hout[:n].copy_(out[:n], non_blocking=True)
+        slot = step % 2
+        done = torch.cuda.Event()
+        done.record(stream)
+        d2h_stream.wait_event(done)
+        with torch.cuda.stream(d2h_stream):
+            houts[slot][:n].copy_(outs[slot][:n], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(d2h_stream)
+        read_done[slot] = ev
+        if read_done[1 - slot] is not None:
+            stream.wait_event(read_done[1 - slot])
         d2h[0] += n * D * 2
 
     cache, queue = new_state()
@@ -382,8 +398,11 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     e0.record(stream)
     if e2e_pool is not None:
         e2e_pool[0].copy_(hpool, non_blocking=True)
-    n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step_e2e, max_steps=args.steps,
-                        cache_all_slots=n_ctx > 1, frame_pool=e2e_pool, fresh_t=fresh_t)
+    n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, outs, H, hd, on_step=on_step_e2e,
+                        max_steps=args.steps, cache_all_slots=n_ctx > 1, frame_pool=e2e_pool, fresh_t=fresh_t)
+    for ev in read_done:
+        if ev is not None:
+            stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)

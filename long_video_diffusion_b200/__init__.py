@@ -576,8 +576,10 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
     own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
-    noise_blocks: device tensors in entry order.  on_step(step, n_win, popped, pushed) is
-    called after each step is enqueued.  max_steps stops the run early (the queue and cache
+    noise_blocks: device tensors in entry order.  out: one output tensor, or a list that the
+    steps use in turn (step s writes out[s % len(out)], e.g. so that a step's output can be
+    read back while the next step runs).  on_step(step, n_win, popped, pushed) is called
+    after each step is enqueued.  max_steps stops the run early (the queue and cache
     are then left mid-run).  cache_all_slots: every step attends to all of the cache ring's
     slots (the last n_slots exited blocks).  frame_pool = (pool, frame_lists): blocks are
     pushed as pool frames (dp_queue_push_frames; the coordinated noise initialisation) and
@@ -614,7 +616,8 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
         nxt = st.nxt
         push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == st.step + 1
         fused_push = push and frame_pool is None
-        window_step(win, win, win, blk, cache, kv_work, out[:n], n_heads, head_dim, pop=pop, queue=queue,
+        o = out[st.step % len(out)] if isinstance(out, (list, tuple)) else out
+        window_step(win, win, win, blk, cache, kv_work, o[:n], n_heads, head_dim, pop=pop, queue=queue,
                     push_noise=noise_blocks[nxt] if fused_push else None, stream=stream, n_win=n,
                     cache_all_slots=cache_all_slots)
         if push and not fused_push:

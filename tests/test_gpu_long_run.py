@@ -124,3 +124,29 @@ def test_long_run_checkpoint_and_resume_is_bit_identical(dp):
     assert cache3.desc.n_advances == cache.desc.n_advances == len(noise) and cache3.length == cache.length
     assert bytes_equal(cache3.k, cache.k) and bytes_equal(cache3.v, cache.v)
     assert queue3.count == queue.count == 0 and queue3.desc.n_popped == queue.desc.n_popped
+
+
+def test_long_run_alternating_output_buffers(dp):
+    """run_fifo with a list of output buffers writes step s into buffer s % 2, with the same
+    values as a run with one buffer."""
+    rc = run_config()
+    H, hd, D, W, T = rc.n_heads, rc.head_dim, rc.hidden, rc.window_blocks, rc.n_timesteps
+    noise = [b.cuda() for b in make_run_noise(rc)]
+    table = make_run_table(rc).cuda()
+    tau = O.timestep_schedule(T)
+    n_max = W * rc.slot_rows
+    kv = torch.empty(2 * n_max * D, dtype=torch.float16, device="cuda")
+    one = torch.empty(n_max, D, dtype=torch.bfloat16, device="cuda")
+    two = [torch.empty_like(one), torch.empty_like(one)]
+    a, b = [], []
+
+    def grab(lst, buf_of):
+        return lambda step, n, popped, pushed: lst.append(buf_of(step)[:n].clone())
+
+    dp.run_fifo(noise, table, tau, W, dp.KVCache(rc.slot_rows, D, torch.float16), dp.Queue(W, rc.slot_rows, D), kv,
+                one, H, hd, on_step=grab(a, lambda s: one), max_steps=60)
+    dp.run_fifo(noise, table, tau, W, dp.KVCache(rc.slot_rows, D, torch.float16), dp.Queue(W, rc.slot_rows, D), kv,
+                two, H, hd, on_step=grab(b, lambda s: two[s % 2]), max_steps=60)
+    dp.device_status()
+    assert len(a) == len(b) == 60
+    assert all(bytes_equal(x, y) for x, y in zip(a, b))
