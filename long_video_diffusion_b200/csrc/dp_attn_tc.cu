@@ -142,7 +142,10 @@ struct Layout {
   // k_full[S], v_full[S], kv_empty[S], q_full[NQ], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ], fin
   static constexpr int N_BAR = 3 * STAGES + 5 * NQ + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  // rows of each stage's key tile that are keys (several-slot instantiation: written by the
+  // producer, read by the softmax warps)
+  static constexpr int OFF_REM = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_REM + STAGES * 4;
   static constexpr int ALLOC = BYTES + 1024;             // room to align the base to 1 KB
   static_assert(ALLOC <= 227 * 1024, "shared memory budget");
 };
@@ -260,10 +263,14 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
         const CUtensorMap* mv = cache ? &tm_vc : &tm_vw;
         int row = (cache ? j : j - p.n_ct) * BN;
         if constexpr (MULTI) {
+          int rem = static_cast<int>(p.n_win - static_cast<int64_t>(j - p.n_ct) * BN);
           if (cache) {
             const int sg = seg_of_tile(sp, j);
             row = pick(sp.seg_row, sg) + (j - pick(sp.seg_tile0, sg)) * BN;
+            rem = pick(sp.seg_len, sg) - (j - pick(sp.seg_tile0, sg)) * BN;
           }
+          // published before the arrive (release) that the softmax's test of k_full acquires
+          reinterpret_cast<volatile int*>(smem + L::OFF_REM)[st] = rem < BN ? rem : BN;
         }
         mbar_arrive_expect_tx(k_full(st), L::KV_BYTES);
 #pragma unroll
@@ -476,10 +483,13 @@ __global__ void __launch_bounds__(Layout<HD>::kThreads, 1)
       const int64_t key0 = (j < p.n_ct) ? static_cast<int64_t>(j) * BN : static_cast<int64_t>(j - p.n_ct) * BN;
       int64_t rem = ((j < p.n_ct) ? p.cache_len : p.n_win) - key0;
       if constexpr (MULTI) {
-        if (j < p.n_ct) {  // rows left in this tile's segment
-          const int sg = seg_of_tile(sp, j);
-          rem = static_cast<int64_t>(pick(sp.seg_len, sg)) - static_cast<int64_t>(j - pick(sp.seg_tile0, sg)) * BN;
-        }
+        // rows of this tile that are keys, as the producer published them for the stage; the
+        // stage's k_full phase for tile j completed before S(j) could (and it is not refilled
+        // before this tile's P is stored), so the test succeeds and orders the read after the
+        // producer's write
+        const int st = j % L::STAGES;
+        if (mbar_test_wait(k_full(st), (j / L::STAGES) & 1))
+          rem = reinterpret_cast<volatile int*>(smem + L::OFF_REM)[st];
       }
       if (rem < BN) {  // last tile of a segment: keys beyond it get -inf (TMA filled them with 0)
         const int valid = static_cast<int>(rem);
