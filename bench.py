@@ -33,8 +33,8 @@ METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 
 # DRAM bytes (read + write) of one attention launch from an ncu capture (summaries under
 # profiles/), valid only for the kernel source they were captured on (md5 over
 # csrc/dp_attn_tc.cu and csrc/dp_device.cuh); any other source reports null.
-TRAFFIC_SOURCE_MD5 = "5c22062a9022bedad07374477645fbd6"
-TRAFFIC_BYTES = {"cogvideo_bf16": 233.452544e6 + 51.196928e6, "wan_bf16": 602.960128e6 + 144.475904e6}
+TRAFFIC_SOURCE_MD5 = "0f4d0a643530e059790321993f0188af"
+TRAFFIC_BYTES = {"cogvideo_bf16": 233.596416e6 + 50.829312e6, "wan_bf16": 633.475072e6 + 142.530048e6}
 L2_BYTES = 126 * 1024 * 1024
 
 
