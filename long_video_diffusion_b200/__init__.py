@@ -472,6 +472,8 @@ def context_refresh(k_ctx, v_ctx, ctx_blocks: DpBlocks, cache: KVCache, stream=N
     """Recompute the context K/V of the window step now (dp_context_refresh): k' = k_ctx *
     (1 + scale_b) + shift_b, v' likewise, written over the cache slot the next step reads;
     k_ctx, v_ctx [n_ctx][hidden] bf16 (f16 cache) or f32 (f32 cache)."""
+    if v_ctx.shape != k_ctx.shape or v_ctx.dtype != k_ctx.dtype:
+        raise ValueError("k_ctx and v_ctx differ in shape or dtype")
     _check(_lib.dp_context_refresh(_ptr(k_ctx), _ptr(v_ctx), k_ctx.shape[0], ctypes.byref(ctx_blocks),
                                    ctypes.byref(cache.desc), _dtype(k_ctx), _stream(k_ctx, stream)),
            "dp_context_refresh")
