@@ -110,6 +110,11 @@ def test_sublayer_fresh_step_matches_oracle(dp, H, hd, n_ctx, t_ctx):
     want, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], fk, fv, n_ctx,
                                  list(np.cumsum([0] + rows)), O.lookup(table, ts), H, hd, EPS, rounded=True)
     assert_close(out.cpu().double().numpy(), want, "bf16", "step over the fresh context")
+    # and against the plain definition: the context's features and the step, nothing rounded
+    pk, pv = O.fresh_context_sublayer(x_ctx, [0, n_ctx], mod_ctx, wts["w_qkv"], wts["b_qkv"], EPS, rounded=False)
+    plain, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], pk, pv, n_ctx,
+                                  list(np.cumsum([0] + rows)), O.lookup(table, ts), H, hd, EPS, rounded=False)
+    assert_close(out.cpu().double().numpy(), plain, "bf16", "step over the fresh context vs the plain definition")
 
 
 # ----------------------------------------------------------------------------- window step

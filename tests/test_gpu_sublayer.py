@@ -5,8 +5,9 @@ against the float64 oracle on the same seeded inputs, through the C ABI.
 Bounds: a 16-bit store of a value v is within one unit in the last place of v (2^-8 |v|
 for bf16, 2^-11 |v| for f16); a fp32 dot product of k terms is within k * 2^-24 times the
 sum of |terms|, at most 2^-12 times it for the k <= 4096 used here.  The whole step is held
-to the bf16 bar of the window step: max-abs 2e-2 and relative L2 5e-3 against the oracle
-that stores its intermediates the same way (h, q, o bf16; k, v f16)."""
+to the bf16 bar of the window step, max-abs 2e-2 and relative L2 5e-3, twice: against the
+plain float64 definition (no intermediate rounded) and against the oracle that stores its
+intermediates where the kernels do (h, q, o bf16; k, v f16)."""
 import numpy as np
 import pytest
 import torch
@@ -86,6 +87,32 @@ def test_qkv_project_splits_q_k_v(dp):
         assert np.all(np.abs(got.cpu().double().numpy() - e) <= unit * np.abs(e) + dot[:, sl] + 1e-7)
 
 
+def test_qkv_project_saturates_k_v_at_the_f16_limit(dp):
+    """k and v leave the projection as f16 features: a value beyond f16's range stores as
+    +-65504 (saturating, not inf).  Large weights push whole columns of k and v past the
+    limit, both signs; q (bf16) keeps the exact value to one bf16 unit."""
+    D, m = 256, 130
+    h = torch.full((m, D), 2.0, dtype=torch.bfloat16)
+    w = torch.zeros(3 * D, D)
+    w[:D] = 0.01
+    w[D:D + 8] = 200.0            # k columns 0..7: 256 * 2 * 200 = 102400
+    w[2 * D:2 * D + 8] = -150.0   # v columns 0..7: -76800
+    w[D + 8:D + 16] = 100.0       # k columns 8..15: 51200, in range
+    w = w.to(torch.bfloat16)
+    q = torch.empty(m, D, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(m, D, dtype=torch.float16, device="cuda")
+    v = torch.empty_like(k)
+    dp.qkv_project(h.cuda(), w.cuda(), None, q, k, v)
+    dp.device_status()
+    exact = O.linear(h, w, None)
+    kg, vg = k.cpu().double().numpy(), v.cpu().double().numpy()
+    assert np.all(np.isfinite(kg)) and np.all(np.isfinite(vg))
+    assert np.all(kg[:, :8] == 65504.0) and np.all(vg[:, :8] == -65504.0)
+    assert np.all(np.abs(kg[:, 8:16] - exact[:, D + 8:D + 16]) <= 2.0 ** -11 * np.abs(exact[:, D + 8:D + 16]))
+    assert np.all(np.abs(q.cpu().double().numpy() - exact[:, :D]) <= 2.0 ** -8 * np.abs(exact[:, :D]) + 1e-6)
+    assert np.array_equal(kg, O.round_to(exact[:, D:2 * D], "f16"))
+
+
 def test_out_project_gated_residual(dp):
     D, rows = 768, [100, 156, 44]
     m = sum(rows)
@@ -136,6 +163,9 @@ def test_sublayer_step_matches_oracle(dp, H, hd, rows, cache_len):
     want, wk, wv = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], ck, cv, cache_len, ro,
                                    mod, H, hd, EPS, rounded=True)
     assert_close(out.cpu().double().numpy(), want, "bf16", "sublayer step")
+    plain, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], ck, cv, cache_len, ro,
+                                  mod, H, hd, EPS, rounded=False)
+    assert_close(out.cpu().double().numpy(), plain, "bf16", "sublayer step vs the plain definition")
     _, q_g, k_g, v_g = dp.sublayer_planes(work, n, D)
     # projected k, v: the GPU's fp32 pre-norm and the oracle's float64 one can round an h
     # element to neighbouring bf16 values (at most one unit, 2^-7 |h|, apart); through W that
@@ -173,6 +203,9 @@ def test_sublayer_step_second_step_uses_the_cache(dp):
     want2, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], cache.k[0].cpu(),
                                   cache.v[0].cpu(), 200, ro, mod, H, hd, EPS, rounded=True)
     assert_close(out2.cpu().double().numpy(), want2, "bf16", "second step")
+    plain2, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], cache.k[0].cpu(),
+                                   cache.v[0].cpu(), 200, ro, mod, H, hd, EPS, rounded=False)
+    assert_close(out2.cpu().double().numpy(), plain2, "bf16", "second step vs the plain definition")
     assert errors(out2.cpu().double().numpy(), out1.cpu().double().numpy())[0] > 1e-3
 
 
@@ -200,6 +233,9 @@ def test_sublayer_step_full_size_sampled(dp):
     want, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], ck, cv, cfg.cache_len,
                                  cfg.row_offset, mod, H, hd, EPS, rounded=True, rows=rows)
     assert_close(out[rows].cpu().double().numpy(), want, "bf16", "cogvideo sublayer")
+    plain, _, _ = O.sublayer_step(x, wts["w_qkv"], wts["b_qkv"], wts["w_o"], wts["b_o"], ck, cv, cfg.cache_len,
+                                  cfg.row_offset, mod, H, hd, EPS, rounded=False, rows=rows)
+    assert_close(out[rows].cpu().double().numpy(), plain, "bf16", "cogvideo sublayer vs the plain definition")
     _, _, k_g, v_g = dp.sublayer_planes(work, n, D)
     n0 = cfg.block_rows[0]
     assert bytes_equal(cache.k[0, :n0], k_g[:n0]) and bytes_equal(cache.v[0, :n0], v_g[:n0])

@@ -1,7 +1,7 @@
 """The shape sweep (16x128 heads, bf16, window 4096..131072 tokens in 4 blocks, cache =
 window/4, random per-block timesteps, a ragged last block variant) through the window step:
-element-by-element against the oracle at the smallest size, sampled rows at the larger
-ones up to the maximum size."""
+element-by-element against the oracle at the smallest size, sampled rows at every larger
+power of two up to the maximum size, each size both regular and ragged (12 cases)."""
 import numpy as np
 import pytest
 import torch
@@ -40,7 +40,8 @@ def test_sweep_4096_full(dp, ragged):
     assert_close(out.cpu().double().numpy(), want, "bf16", cfg.name)
 
 
-@pytest.mark.parametrize("n,ragged", [(16384, True), (65536, False), (131072, False), (131072, True)])
+@pytest.mark.parametrize("n", [8192, 16384, 32768, 65536, 131072])
+@pytest.mark.parametrize("ragged", [False, True], ids=["regular", "ragged"])
 def test_sweep_sampled(dp, n, ragged):
     cfg = step_config("sweep", n, ragged=ragged)
     x, out = _run(dp, cfg)
