@@ -15,6 +15,8 @@
  *       prologue and the gate (+ residual) into its epilogue   dp_window_attention
  *   A3  queue and cache advance               dp_kvcache_advance, dp_queue_push/pop
  *   A4  the whole step A1 -> A2 -> A3         dp_window_step
+ *   the queue's schedule over a whole video (host) and the coordinated noise
+ *   initialisation's frame selection: dp_fifo_*, dp_coordinated_frames
  *   B   the DiT attention sublayer around A2 (pre-norm, q/k/v and output projections on
  *       caller-supplied weights): dp_ln_modulate, dp_linear, dp_qkv_project,
  *       dp_out_project, dp_sublayer_step
@@ -212,8 +214,8 @@ dp_status dp_queue_push(dp_queue* q, const void* noise, int64_t rows, void* stre
  * that concatenated blocks do not repeat noise): the pushed block is the concatenation of
  * frames frame_idx[0 .. n_frames) (host array) of pool (DEVICE [pool_frames][frame_rows]
  * [hidden], the queue's type), written to the queue's tail slot like dp_queue_push (byte
- * copy, bit-exact).  Which frames (the shuffle) is the caller's choice; the binding's
- * coordinated_frames() implements the selection rule.  n_frames in [1, 16] (UNSUPPORTED
+ * copy, bit-exact).  Which frames (the shuffle) is the caller's choice;
+ * dp_coordinated_frames implements the selection rule.  n_frames in [1, 16] (UNSUPPORTED
  * otherwise); INVALID_ARG for an index outside [0, pool_frames); CAPACITY as dp_queue_push
  * for n_frames * frame_rows rows. */
 dp_status dp_queue_push_frames(dp_queue* q, const void* pool, int32_t pool_frames,
@@ -222,6 +224,79 @@ dp_status dp_queue_push_frames(dp_queue* q, const void* pool, int32_t pool_frame
 
 /* Pop the head block (metadata only: the slot becomes free).  EMPTY if no block. */
 dp_status dp_queue_pop(dp_queue* q);
+
+/* ---------------------------------------------------------------- the queue's schedule (host) */
+
+/*
+ * The FIFO schedule of a whole video (the review's key machinery and its Figure 1: blocks
+ * enter at the tail one after another, every live block is evaluated once per step at its
+ * own timestep, and a block leaves at the head after its last evaluation).  Block b enters
+ * at step e_b = floor(b * T / W): with T evaluations per block and W blocks in the
+ * steady-state window this gives exactly W live blocks in the steady state, T evaluations
+ * of every block, and the exit of block b in the same step as the entry of block b + W
+ * (the pages give no stagger; this is the plainest one with those properties).  The video
+ * has n_blocks blocks; the run ends after step e_{n_blocks-1} + T - 1.  T >= W >= 1 (at
+ * most one block enters per step), W <= DP_MAX_SLOTS.  Host plain data; the library
+ * updates it in dp_fifo_commit.
+ */
+typedef struct {
+  int32_t n_blocks;       /* blocks in the whole video */
+  int32_t n_timesteps;    /* T: evaluations per block */
+  int32_t window_blocks;  /* W: live blocks in the steady state */
+  int32_t next_block;     /* the next block to enter (0: none has entered yet) */
+  int64_t step;           /* schedule steps taken */
+  int64_t exited_rows;    /* rows of the block that left last (0 before the first exit) */
+} dp_fifo;
+
+/* What one step of the schedule does, as dp_fifo_plan computes it. */
+typedef struct {
+  int32_t push_before;    /* block to push before the step (block 0 at step 0), else -1 */
+  int32_t pop;            /* 1: the head block has its last evaluation in this step and
+                             exits after it (DP_STEP_POP) */
+  int32_t push_after;     /* block that enters after this step (pushed with or after it), else -1 */
+  int32_t done;           /* 1: every block has left; there is no step to take */
+  int64_t exit_rows;      /* rows of the head block when pop = 1, else 0 */
+  const void* ctx_rows;   /* DEVICE address of the latent rows of the block that left last,
+                             while the queue still holds them in the slot behind its head
+                             (a queue with more slots than W), else NULL: the rows a fresh
+                             context is recomputed from */
+  int64_t ctx_n;          /* their row count (0 with ctx_rows NULL) */
+} dp_fifo_step;
+
+/* Entry step of block b: *step = floor(b * T / W).  INVALID_ARG unless b >= 0 and
+ * T >= W >= 1. */
+dp_status dp_fifo_entry_step(int32_t b, int32_t n_timesteps, int32_t window_blocks, int64_t* step);
+
+/* A fresh schedule of n_blocks blocks (step 0, no block entered).  INVALID_ARG unless
+ * n_blocks >= 1 and T >= W with 1 <= W <= DP_MAX_SLOTS. */
+dp_status dp_fifo_init(dp_fifo* f, int32_t n_blocks, int32_t n_timesteps, int32_t window_blocks);
+
+/* The next step of the schedule f for the queue q (host descriptor; its state after
+ * push_before is what the step sees): whether the head block exits after the step, which
+ * block enters, and the rows of the block that left last.  The queue must match the
+ * schedule (its live count and its head block's evaluation count at this step, counting
+ * push_before), else INVALID_ARG; done = 1 once every block has left.  Reads q only. */
+dp_status dp_fifo_plan(const dp_fifo* f, const dp_queue* q, dp_fifo_step* out);
+
+/* Record that the planned step ran (and its pushes were made): step += 1, next_block moves
+ * past push_before and push_after, exited_rows = exit_rows when pop.  INVALID_ARG if the
+ * plan is not the schedule's next step. */
+dp_status dp_fifo_commit(dp_fifo* f, const dp_fifo_step* s);
+
+/* Coordinated noise initialisation, the frame selection (the abstract: initial noise
+ * patterns shared at no extra cost; the review: a full noise pool, shuffled assignment,
+ * the last latents excluded).  The pool is the first window: the frames of blocks
+ * 0 .. W-1, pool_frames = block_frames[0] + ... + block_frames[W-1] (W = min(window_blocks,
+ * n_blocks)).  Block b < W takes its own frames of the pool in order; block b >= W takes
+ * the pool frames in the order of perm (host, a permutation of [0, pool_frames), drawn by
+ * the caller), skipping prev_frames (host, n_prev frames: the block just before it), the
+ * first block_frames[b] of them.  frames_out (host) receives block_frames[b] pool frame
+ * indices.  INVALID_ARG if perm is not a permutation (for b >= W), b is outside
+ * [0, n_blocks), or the pool holds fewer than block_frames[b] frames outside prev_frames;
+ * the result goes to dp_queue_push_frames. */
+dp_status dp_coordinated_frames(const int32_t* block_frames, int32_t n_blocks, int32_t window_blocks,
+                                int32_t b, const int32_t* prev_frames, int32_t n_prev,
+                                const int32_t* perm, int32_t* frames_out);
 
 /* ---------------------------------------------------------------- A4: window step */
 
@@ -261,8 +336,10 @@ dp_status dp_window_step(const void* q, const void* k, const void* v, int64_t n_
  * library's device memory, held by every device that loads the library until the process
  * exits.  The call allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  * CAPACITY, before anything is enqueued, if 2 * n_win * n_heads * head_dim feature
- * elements (2 bytes each for bf16 windows, 4 for fp32) exceed that size.  The first call on
- * a device looks up the array's device address (cudaGetSymbolAddress, with that device
+ * elements (2 bytes each for bf16 windows, 4 for fp32) exceed that size (the sizes are
+ * compared without forming the product, so no size overflows).  The first call on a
+ * device, and the first after a device reset (a new CUDA context, recognised by its
+ * context id), looks up the array's device address (cudaGetSymbolAddress, with that device
  * current); make that first call before any stream capture.  All calls share the one
  * array: calls whose work overlaps on the GPU (other streams, other threads) race on it;
  * order them on one stream.  Its contents from earlier calls are never read (the

@@ -64,6 +64,17 @@ class DpQueue(ctypes.Structure):
                 ("n_pushed", ctypes.c_int64), ("n_popped", ctypes.c_int64), ("dtype", ctypes.c_int32)]
 
 
+class DpFifo(ctypes.Structure):
+    _fields_ = [("n_blocks", ctypes.c_int32), ("n_timesteps", ctypes.c_int32), ("window_blocks", ctypes.c_int32),
+                ("next_block", ctypes.c_int32), ("step", ctypes.c_int64), ("exited_rows", ctypes.c_int64)]
+
+
+class DpFifoStep(ctypes.Structure):
+    _fields_ = [("push_before", ctypes.c_int32), ("pop", ctypes.c_int32), ("push_after", ctypes.c_int32),
+                ("done", ctypes.c_int32), ("exit_rows", ctypes.c_int64), ("ctx_rows", ctypes.c_void_p),
+                ("ctx_n", ctypes.c_int64)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _U32, _F = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float
 _SIGS = {
@@ -78,6 +89,12 @@ _SIGS = {
     "dp_queue_push": [ctypes.POINTER(DpQueue), _P, _I64, _P],
     "dp_queue_pop": [ctypes.POINTER(DpQueue)],
     "dp_queue_push_frames": [ctypes.POINTER(DpQueue), _P, _I32, _I64, ctypes.POINTER(_I32), _I32, _P],
+    "dp_fifo_entry_step": [_I32, _I32, _I32, ctypes.POINTER(_I64)],
+    "dp_fifo_init": [ctypes.POINTER(DpFifo), _I32, _I32, _I32],
+    "dp_fifo_plan": [ctypes.POINTER(DpFifo), ctypes.POINTER(DpQueue), ctypes.POINTER(DpFifoStep)],
+    "dp_fifo_commit": [ctypes.POINTER(DpFifo), ctypes.POINTER(DpFifoStep)],
+    "dp_coordinated_frames": [ctypes.POINTER(_I32), _I32, _I32, _I32, ctypes.POINTER(_I32), _I32,
+                              ctypes.POINTER(_I32), ctypes.POINTER(_I32)],
     "dp_window_step": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P, _P,
                        _I32, _I32, _U32, ctypes.POINTER(DpQueue), _P, _I64, _I32, _P],
     "dp_window_step_noalloc": [_P, _P, _P, _I64, ctypes.POINTER(DpBlocks), ctypes.POINTER(DpKvcache), _P, _P,
@@ -298,19 +315,31 @@ def queue_push_frames(queue: Queue, pool: torch.Tensor, frames: Sequence[int], s
                                      len(frames), _stream(queue.latent, stream)), "dp_queue_push_frames")
 
 
-def coordinated_frames(pool_frames: int, block_frames: int, prev_frames: Sequence[int],
-                       perm: Sequence[int]) -> list:
-    """Frames of a new block under the coordinated noise initialisation: the pool's frames in
-    the order of the random permutation perm, without the frames the previous block used
-    (adjacent blocks share no noise frame), the first block_frames of them."""
-    prev = set(int(f) for f in prev_frames)
-    out = []
-    for f in perm:
-        if int(f) not in prev:
-            out.append(int(f))
-            if len(out) == block_frames:
-                return out
-    raise ValueError("the pool has too few frames outside the previous block")
+def coordinated_frames(block_frames: Sequence[int], window_blocks: int, b: int, prev_frames: Sequence[int],
+                       perm: Optional[Sequence[int]]) -> list:
+    """Pool frames of block b under the coordinated noise initialisation
+    (dp_coordinated_frames): the pool is the first window's frames; block b < window_blocks
+    takes its own frames in order, a later block the pool's frames in the order of the random
+    permutation perm without prev_frames (the block before it)."""
+    n = len(block_frames)
+    bf = (_I32 * n)(*[int(f) for f in block_frames])
+    prev = (_I32 * max(1, len(prev_frames)))(*[int(f) for f in prev_frames])
+    pm = None if perm is None else (_I32 * len(perm))(*[int(f) for f in perm])
+    nf = int(block_frames[b]) if 0 <= b < n else 1
+    out = (_I32 * max(1, nf))()
+    _check(_lib.dp_coordinated_frames(bf, n, int(window_blocks), int(b), prev, len(prev_frames), pm, out),
+           "dp_coordinated_frames")
+    return [out[i] for i in range(nf)]
+
+
+def coordinated_schedule(block_frames: Sequence[int], window_blocks: int, perms) -> list:
+    """Pool frames of every block of a video, block b from perms[b] (dp_coordinated_frames
+    block after block)."""
+    lists: list = []
+    for b in range(len(block_frames)):
+        lists.append(coordinated_frames(block_frames, window_blocks, b, lists[b - 1] if b else [],
+                                        perms[b] if b >= window_blocks else None))
+    return lists
 
 
 def queue_pop(queue: Queue) -> None:
@@ -526,12 +555,13 @@ def profile_end_stages(max_stages: int = 5):
     return [ms[i] for i in range(max_stages)], ns.value, n.value
 
 
-NOALLOC_SCRATCH_BYTES = 32 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20   # DP_NOALLOC_SCRATCH_BYTES of include/dp.h (a CPU test keeps them equal)
 
 
 def window_step_noalloc(q, k, v, blocks: DpBlocks, cache: KVCache, out, n_heads: int, head_dim: int,
                         pop: bool = False, queue: Optional[Queue] = None, push_noise=None, push_rows=None,
-                        residual=None, stream=None, n_win: Optional[int] = None) -> None:
+                        residual=None, stream=None, n_win: Optional[int] = None,
+                        cache_all_slots: bool = False) -> None:
     """window_step without kv_work, for callers that cannot allocate device memory: the
     k'/v' scratch is a fixed NOALLOC_SCRATCH_BYTES array inside the library (see
     dp_window_step_noalloc).  Calls share that array, so they must not overlap on the GPU."""
@@ -545,7 +575,8 @@ def window_step_noalloc(q, k, v, blocks: DpBlocks, cache: KVCache, out, n_heads:
         qp, kp, vp = ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v)
     rows = 0 if push_noise is None else (push_noise.shape[0] if push_rows is None else push_rows)
     _check(_lib.dp_window_step_noalloc(qp, kp, vp, n, ctypes.byref(blocks), ctypes.byref(cache.desc),
-                                       _ptr(residual), _ptr(out), n_heads, head_dim, STEP_POP if pop else 0,
+                                       _ptr(residual), _ptr(out), n_heads, head_dim,
+                                       (STEP_POP if pop else 0) | (STEP_CACHE_ALL_SLOTS if cache_all_slots else 0),
                                        ctypes.byref(queue.desc) if queue is not None else None,
                                        _ptr(push_noise), int(rows), _dtype(out), _stream(ref, stream)),
            "dp_window_step_noalloc")
@@ -566,9 +597,11 @@ def loaded_library_path() -> str:
 # ------------------------------------------------------------------------- long-video run
 
 def fifo_entry_step(b: int, n_timesteps: int, window_blocks: int) -> int:
-    """Step at which block b enters the queue: floor(b * T / W), so that the window holds W
-    blocks in steady state and block b's exit coincides with block b + W's entry."""
-    return (b * n_timesteps) // window_blocks
+    """Step at which block b enters the queue (dp_fifo_entry_step)."""
+    out = _I64()
+    _check(_lib.dp_fifo_entry_step(int(b), int(n_timesteps), int(window_blocks), ctypes.byref(out)),
+           "dp_fifo_entry_step")
+    return out.value
 
 
 def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_blocks: int, cache: KVCache,
@@ -577,68 +610,85 @@ def run_fifo(noise_blocks, table: torch.Tensor, tau: Sequence[int], window_block
              frame_pool=None, fresh_t: Optional[int] = None, state: Optional["FifoState"] = None) -> int:
     """Denoise a whole video through the block queue (the pages' FIFO: push a noisy block at
     the tail, pop a clean block at the head; every block is evaluated once per step at its
-    own timestep tau[evals]).  q = k = v = the queue's live window (identity projections).
-    noise_blocks: device tensors in entry order.  out: one output tensor, or a list that the
-    steps use in turn (step s writes out[s % len(out)], e.g. so that a step's output can be
-    read back while the next step runs).  on_step(step, n_win, popped, pushed) is called
-    after each step is enqueued.  max_steps stops the run early (the queue and cache
-    are then left mid-run).  cache_all_slots: every step attends to all of the cache ring's
-    slots (the last n_slots exited blocks).  frame_pool = (pool, frame_lists): blocks are
-    pushed as pool frames (dp_queue_push_frames; the coordinated noise initialisation) and
-    noise_blocks only gives each block's row count.  fresh_t: before every step after the
-    first exit, the context K/V are recomputed (dp_context_refresh) from the latent rows of
-    the block that left last, conditioned on table[fresh_t], instead of reused from its last
-    evaluation; the queue keeps those rows in the slot behind its head, so it needs more
-    slots than window_blocks.  state: the run's progress (FifoState), updated as steps are
-    enqueued; a run stopped by max_steps continues from it, also after checkpoint/restore.
-    Returns the number of steps run so far (state.step)."""
+    own timestep tau[evals]).  The schedule (which block enters when, when the head exits)
+    is the library's (dp_fifo_plan / dp_fifo_commit); this loop only carries out its steps.
+    q = k = v = the queue's live window (identity projections).  noise_blocks: device
+    tensors in entry order.  out: one output tensor, or a list that the steps use in turn
+    (step s writes out[s % len(out)], e.g. so that a step's output can be read back while
+    the next step runs).  on_step(step, n_win, popped, pushed) is called after each step is
+    enqueued.  max_steps stops the run early (the queue and cache are then left mid-run).
+    cache_all_slots: every step attends to all of the cache ring's slots (the last n_slots
+    exited blocks).  frame_pool = (pool, frame_lists): blocks are pushed as pool frames
+    (dp_queue_push_frames; the coordinated noise initialisation) and noise_blocks only gives
+    each block's row count.  fresh_t: before every step after the first exit, the context
+    K/V are recomputed (dp_context_refresh) from the latent rows of the block that left last,
+    conditioned on table[fresh_t], instead of reused from its last evaluation; the queue
+    keeps those rows in the slot behind its head, so it needs more slots than
+    window_blocks.  state: the run's progress (FifoState), updated as steps are enqueued; a
+    run stopped by max_steps continues from it, also after checkpoint/restore.  Returns the
+    number of steps run so far (state.step)."""
     T = len(tau)
     n_blocks = len(noise_blocks)
     if fresh_t is not None and queue.desc.n_slots <= window_blocks:
         raise ValueError("a fresh context needs a queue with more slots than window blocks")
     st = state if state is not None else FifoState()
+    st.bind(n_blocks, T, window_blocks)
+    plan = DpFifoStep()
+    lat = queue.latent
+
     def push_block(b):
         if frame_pool is None:
             queue_push(queue, noise_blocks[b], stream=stream)
         else:
             queue_push_frames(queue, frame_pool[0], frame_pool[1][b], stream=stream)
 
-    if st.nxt == 0:
-        push_block(0)
-        st.nxt = 1
     run = 0
-    while queue.count > 0 and (max_steps is None or run < max_steps):
-        if fresh_t is not None and st.exited_rows > 0:
-            ctx = queue.latent[(queue.head - 1) % queue.desc.n_slots, :st.exited_rows]
-            context_refresh(ctx, ctx, blocks_from_table(table, [fresh_t], [st.exited_rows]), cache, stream=stream)
+    while max_steps is None or run < max_steps:
+        _check(_lib.dp_fifo_plan(ctypes.byref(st.desc), ctypes.byref(queue.desc), ctypes.byref(plan)), "dp_fifo_plan")
+        if plan.done:
+            break
+        if plan.push_before >= 0:
+            push_block(plan.push_before)
+            _check(_lib.dp_fifo_commit(ctypes.byref(st.desc), ctypes.byref(plan)), "dp_fifo_commit")
+            continue
+        if fresh_t is not None and plan.ctx_rows:
+            first = (plan.ctx_rows - lat.data_ptr()) // lat.element_size()
+            ctx = lat.view(-1)[first:first + plan.ctx_n * lat.shape[2]].view(plan.ctx_n, lat.shape[2])
+            context_refresh(ctx, ctx, blocks_from_table(table, [fresh_t], [plan.ctx_n]), cache, stream=stream)
         blk, win, n = queue_blocks(queue, table, tau)
-        pop = queue.evals()[0] + 1 == T
-        if pop:
-            st.exited_rows = queue.rows()[0]
-        nxt = st.nxt
-        push = nxt < n_blocks and fifo_entry_step(nxt, T, window_blocks) == st.step + 1
-        fused_push = push and frame_pool is None
+        push = plan.push_after if plan.push_after >= 0 else None
+        fused_push = push is not None and frame_pool is None
         o = out[st.step % len(out)] if isinstance(out, (list, tuple)) else out
-        window_step(win, win, win, blk, cache, kv_work, o[:n], n_heads, head_dim, pop=pop, queue=queue,
-                    push_noise=noise_blocks[nxt] if fused_push else None, stream=stream, n_win=n,
+        window_step(win, win, win, blk, cache, kv_work, o[:n], n_heads, head_dim, pop=bool(plan.pop), queue=queue,
+                    push_noise=noise_blocks[push] if fused_push else None, stream=stream, n_win=n,
                     cache_all_slots=cache_all_slots)
-        if push and not fused_push:
-            push_block(nxt)
+        if push is not None and not fused_push:
+            push_block(push)
         if on_step is not None:
-            on_step(st.step, n, pop, nxt if push else None)
-        if push:
-            st.nxt += 1
-        st.step += 1
+            on_step(st.step, n, bool(plan.pop), push)
+        _check(_lib.dp_fifo_commit(ctypes.byref(st.desc), ctypes.byref(plan)), "dp_fifo_commit")
         run += 1
     return st.step
 
 
 class FifoState:
-    """Progress of a run_fifo run: steps taken, the next block to push (0 = none pushed yet)
-    and the row count of the block that left last."""
+    """Progress of a run_fifo run (the library's dp_fifo schedule): steps taken, the next
+    block to push (0 = none pushed yet) and the row count of the block that left last."""
 
     def __init__(self, step: int = 0, nxt: int = 0, exited_rows: int = 0):
-        self.step, self.nxt, self.exited_rows = step, nxt, exited_rows
+        self.desc = DpFifo()
+        self.desc.step, self.desc.next_block, self.desc.exited_rows = step, nxt, exited_rows
+
+    def bind(self, n_blocks: int, n_timesteps: int, window_blocks: int) -> None:
+        """Attach the schedule's sizes (dp_fifo_init for a fresh run, the saved progress kept)."""
+        step, nxt, ex = self.step, self.nxt, self.exited_rows
+        _check(_lib.dp_fifo_init(ctypes.byref(self.desc), int(n_blocks), int(n_timesteps), int(window_blocks)),
+               "dp_fifo_init")
+        self.desc.step, self.desc.next_block, self.desc.exited_rows = step, nxt, ex
+
+    step = property(lambda self: self.desc.step)
+    nxt = property(lambda self: self.desc.next_block)
+    exited_rows = property(lambda self: self.desc.exited_rows)
 
 
 _QUEUE_FIELDS = ("slot_rows", "hidden", "n_slots", "head", "count", "n_pushed", "n_popped", "dtype")

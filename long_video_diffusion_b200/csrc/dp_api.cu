@@ -980,4 +980,175 @@ dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, c
   return DP_OK;
 }
 
+// ------------------------------------------------------------------ the queue's schedule (host)
+
+namespace {
+
+// floor(b * T / W): entry step of block b (the review's Figure 1 stagger, made exact).
+int64_t entry_step(int64_t b, int32_t T, int32_t W) { return b * T / W; }
+
+dp_status check_fifo(const dp_fifo* f) {
+  if (!f) return fail(DP_ERR_INVALID_ARG, "schedule is NULL");
+  if (f->n_blocks < 1 || f->window_blocks < 1 || f->window_blocks > DP_MAX_SLOTS ||
+      f->n_timesteps < f->window_blocks)
+    return fail(DP_ERR_INVALID_ARG, "schedule: n_blocks %d, T %d, W %d (need n_blocks >= 1, T >= W, 1 <= W <= %d)",
+                f->n_blocks, f->n_timesteps, f->window_blocks, DP_MAX_SLOTS);
+  if (f->next_block < 0 || f->next_block > f->n_blocks || f->step < 0 || f->exited_rows < 0)
+    return fail(DP_ERR_INVALID_ARG, "schedule state: next_block %d, step %lld", f->next_block,
+                static_cast<long long>(f->step));
+  return DP_OK;
+}
+
+}  // namespace
+
+dp_status dp_fifo_entry_step(int32_t b, int32_t n_timesteps, int32_t window_blocks, int64_t* step) {
+  if (!step || b < 0 || window_blocks < 1 || n_timesteps < window_blocks)
+    return fail(DP_ERR_INVALID_ARG, "entry step of block %d with T %d, W %d", b, n_timesteps, window_blocks);
+  *step = entry_step(b, n_timesteps, window_blocks);
+  return DP_OK;
+}
+
+dp_status dp_fifo_init(dp_fifo* f, int32_t n_blocks, int32_t n_timesteps, int32_t window_blocks) {
+  if (!f) return fail(DP_ERR_INVALID_ARG, "schedule is NULL");
+  dp_fifo g;
+  g.n_blocks = n_blocks;
+  g.n_timesteps = n_timesteps;
+  g.window_blocks = window_blocks;
+  g.next_block = 0;
+  g.step = 0;
+  g.exited_rows = 0;
+  dp_status st = check_fifo(&g);
+  if (st != DP_OK) return st;
+  *f = g;
+  return DP_OK;
+}
+
+dp_status dp_fifo_plan(const dp_fifo* f, const dp_queue* q, dp_fifo_step* out) {
+  dp_status st = check_fifo(f);
+  if (st != DP_OK) return st;
+  if (!q || !out) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  st = check_queue(q, q->hidden, q->dtype);
+  if (st != DP_OK) return st;
+  const int32_t T = f->n_timesteps, W = f->window_blocks;
+  const int64_t s = f->step;
+  dp_fifo_step o;
+  o.push_before = -1;
+  o.pop = 0;
+  o.push_after = -1;
+  o.done = 0;
+  o.exit_rows = 0;
+  o.ctx_rows = nullptr;
+  o.ctx_n = 0;
+  const int64_t total = entry_step(f->n_blocks - 1, T, W) + T;  // steps of the whole run
+  if (s >= total) {
+    if (q->count != 0 || f->next_block != f->n_blocks)
+      return fail(DP_ERR_INVALID_ARG, "schedule finished but the queue holds %d blocks", q->count);
+    o.done = 1;
+    *out = o;
+    return DP_OK;
+  }
+  if (f->next_block == 0) {
+    // block 0 enters before step 0: the caller pushes it, commits, and plans again
+    if (s != 0 || q->count != 0) return fail(DP_ERR_INVALID_ARG, "no block entered but step %lld, queue %d",
+                                             static_cast<long long>(s), q->count);
+    o.push_before = 0;
+    *out = o;
+    return DP_OK;
+  }
+  // live blocks at step s: [lo, hi), e_b <= s < e_b + T
+  int64_t lo = 0;
+  while (lo < f->n_blocks && entry_step(lo, T, W) + T <= s) ++lo;
+  int64_t hi = lo;
+  while (hi < f->n_blocks && entry_step(hi, T, W) <= s) ++hi;
+  if (hi != f->next_block || q->count != hi - lo)
+    return fail(DP_ERR_INVALID_ARG, "queue does not match the schedule at step %lld: %d live blocks, %lld expected "
+                "(blocks %lld..%lld entered, next %d)", static_cast<long long>(s), q->count,
+                static_cast<long long>(hi - lo), static_cast<long long>(lo), static_cast<long long>(hi - 1),
+                f->next_block);
+  if (q->count < 1 || q->evals[0] != s - entry_step(lo, T, W))
+    return fail(DP_ERR_INVALID_ARG, "head block has %d evaluations at step %lld, %lld expected", q->evals[0],
+                static_cast<long long>(s), static_cast<long long>(s - entry_step(lo, T, W)));
+  o.pop = (s - entry_step(lo, T, W) == T - 1) ? 1 : 0;
+  o.exit_rows = o.pop ? q->rows[0] : 0;
+  if (f->next_block < f->n_blocks && entry_step(f->next_block, T, W) == s + 1) o.push_after = f->next_block;
+  // the block that left last keeps its rows in the slot behind the head until a push reuses
+  // it, which cannot happen while the queue has more slots than live blocks
+  if (f->exited_rows > 0 && q->n_slots > W) {
+    o.ctx_rows = queue_slot(q, (q->head + q->n_slots - 1) % q->n_slots);
+    o.ctx_n = f->exited_rows;
+  }
+  *out = o;
+  return DP_OK;
+}
+
+dp_status dp_fifo_commit(dp_fifo* f, const dp_fifo_step* s) {
+  dp_status st = check_fifo(f);
+  if (st != DP_OK) return st;
+  if (!s) return fail(DP_ERR_INVALID_ARG, "step is NULL");
+  if (s->done) return fail(DP_ERR_INVALID_ARG, "the schedule is finished");
+  if (s->push_before >= 0) {
+    if (s->push_before != 0 || f->next_block != 0 || f->step != 0)
+      return fail(DP_ERR_INVALID_ARG, "push_before %d is not the schedule's first push", s->push_before);
+    f->next_block = 1;
+    return DP_OK;
+  }
+  if (f->next_block == 0) return fail(DP_ERR_INVALID_ARG, "block 0 has not entered");
+  if (s->push_after >= 0 &&
+      (s->push_after != f->next_block || f->next_block >= f->n_blocks ||
+       entry_step(f->next_block, f->n_timesteps, f->window_blocks) != f->step + 1))
+    return fail(DP_ERR_INVALID_ARG, "push_after %d is not the block entering after step %lld", s->push_after,
+                static_cast<long long>(f->step));
+  if (s->push_after < 0 && f->next_block < f->n_blocks &&
+      entry_step(f->next_block, f->n_timesteps, f->window_blocks) == f->step + 1)
+    return fail(DP_ERR_INVALID_ARG, "block %d enters after step %lld but the plan pushes none", f->next_block,
+                static_cast<long long>(f->step));
+  if (s->pop && s->exit_rows <= 0) return fail(DP_ERR_INVALID_ARG, "pop of an empty block");
+  f->step += 1;
+  if (s->push_after >= 0) f->next_block += 1;
+  if (s->pop) f->exited_rows = s->exit_rows;
+  return DP_OK;
+}
+
+// ------------------------------------------------------------------ coordinated noise initialisation
+
+dp_status dp_coordinated_frames(const int32_t* block_frames, int32_t n_blocks, int32_t window_blocks, int32_t b,
+                                const int32_t* prev_frames, int32_t n_prev, const int32_t* perm,
+                                int32_t* frames_out) {
+  if (!block_frames || !frames_out || n_blocks < 1 || window_blocks < 1 || b < 0 || b >= n_blocks || n_prev < 0 ||
+      (n_prev > 0 && !prev_frames))
+    return fail(DP_ERR_INVALID_ARG, "coordinated frames: block %d of %d, W %d, %d previous frames", b, n_blocks,
+                window_blocks, n_prev);
+  const int32_t W = window_blocks < n_blocks ? window_blocks : n_blocks;
+  int64_t pool = 0, first = 0;
+  for (int32_t i = 0; i < W; ++i) {
+    if (block_frames[i] < 1) return fail(DP_ERR_INVALID_ARG, "block %d has %d frames", i, block_frames[i]);
+    if (i < b) first += block_frames[i];
+    pool += block_frames[i];
+  }
+  if (pool > (1 << 24)) return fail(DP_ERR_INVALID_ARG, "pool of %lld frames", static_cast<long long>(pool));
+  const int32_t nf = block_frames[b];
+  if (nf < 1) return fail(DP_ERR_INVALID_ARG, "block %d has %d frames", b, nf);
+  if (b < W) {
+    // the first window is the pool itself, in order
+    for (int32_t i = 0; i < nf; ++i) frames_out[i] = static_cast<int32_t>(first + i);
+    return DP_OK;
+  }
+  if (!perm) return fail(DP_ERR_INVALID_ARG, "perm is NULL");
+  // perm must hold every pool frame once; prev_frames are excluded
+  std::vector<uint8_t> seen(static_cast<size_t>(pool), 0), excluded(static_cast<size_t>(pool), 0);
+  for (int64_t i = 0; i < pool; ++i) {
+    const int32_t f = perm[i];
+    if (f < 0 || f >= pool || seen[f]) return fail(DP_ERR_INVALID_ARG, "perm is not a permutation of the pool");
+    seen[f] = 1;
+  }
+  for (int32_t i = 0; i < n_prev; ++i)
+    if (prev_frames[i] >= 0 && prev_frames[i] < pool) excluded[prev_frames[i]] = 1;
+  int32_t got = 0;
+  for (int64_t i = 0; i < pool && got < nf; ++i)
+    if (!excluded[perm[i]]) frames_out[got++] = perm[i];
+  if (got < nf)
+    return fail(DP_ERR_INVALID_ARG, "the pool has %d frames outside the previous block, %d needed", got, nf);
+  return DP_OK;
+}
+
 }  // extern "C"

@@ -7,6 +7,7 @@
 // cudaMalloc/cudaFree would synchronize the device.  This entry point takes the same
 // arguments minus kv_work and uses a fixed array in the library's own device memory
 // instead.  It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -24,24 +25,64 @@ namespace {
 static __device__ __align__(256) unsigned char g_step_scratch[DP_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+
+// The array's address, per device, valid for the CUDA context it was looked up in.  A
+// device reset destroys that context (and the module's copy of the array with it); the
+// context that replaces it has a new id, so the address is looked up again.
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;  // 0: not looked up yet
+  void* addr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Set-up, once per device, with that device current: the device address of the array.
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+template <class F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+
+// Unique id of the calling thread's current context (0 if there is none yet).
+bool current_ctx_id(unsigned long long* id) {
+  static PfnCtxGetCurrent get_current = driver_fn<PfnCtxGetCurrent>("cuCtxGetCurrent");
+  static PfnCtxGetId get_id = driver_fn<PfnCtxGetId>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  if (ctx == nullptr) return true;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// The device address of the array on the current device.  Set-up, once per device and
+// context, with that device current: cudaGetSymbolAddress (which also makes the runtime's
+// context current if the thread had none).  Later calls compare the context id only.
 dp_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return dp::set_error(DP_ERR_CUDA, "cudaGetDevice failed");
   if (dev < 0 || dev >= kMaxDevices) return dp::set_error(DP_ERR_UNSUPPORTED, "device ordinal out of range");
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  unsigned long long id = 0;
+  if (!current_ctx_id(&id)) return dp::set_error(DP_ERR_CUDA, "cannot read the current CUDA context");
+  ScratchSlot& slot = g_scratch[dev];
+  if (id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_step_scratch);
     if (e != cudaSuccess || p == nullptr)
       return dp::set_error(DP_ERR_CUDA, "cudaGetSymbolAddress of the step scratch failed");
-    g_scratch_addr[dev] = p;
+    if (!current_ctx_id(&id) || id == 0) return dp::set_error(DP_ERR_CUDA, "no current CUDA context after set-up");
+    slot.ctx_id = id;
+    slot.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return DP_OK;
 }
 
@@ -54,14 +95,18 @@ extern "C" dp_status dp_window_step_noalloc(const void* q, const void* k, const 
                                             void* stream) {
   if (n_win <= 0 || n_heads <= 0 || head_dim <= 0)
     return dp::set_error(DP_ERR_INVALID_ARG, "n_win, n_heads and head_dim must be positive");
-  // k' and v' of the window, in the feature type (f16 for bf16 windows, fp32 for fp32)
+  // k' and v' of the window, in the feature type (f16 for bf16 windows, fp32 for fp32):
+  // 2 * n_win * hidden elements.  Compared by division, so no product can overflow.
   const uint64_t feat_bytes = dt == DP_F32 ? 4u : 2u;
-  const uint64_t need = 2ull * static_cast<uint64_t>(n_win) * static_cast<uint64_t>(n_heads) *
-                        static_cast<uint64_t>(head_dim) * feat_bytes;
-  if (need > DP_NOALLOC_SCRATCH_BYTES) {
-    char msg[160];
-    snprintf(msg, sizeof(msg), "window needs %llu scratch bytes; the fixed scratch holds %llu",
-             static_cast<unsigned long long>(need), static_cast<unsigned long long>(DP_NOALLOC_SCRATCH_BYTES));
+  const uint64_t limit = DP_NOALLOC_SCRATCH_BYTES;
+  const uint64_t hidden = static_cast<uint64_t>(n_heads) * static_cast<uint64_t>(head_dim);
+  const uint64_t row_bytes = hidden <= limit ? 2u * hidden * feat_bytes : limit + 1;
+  if (row_bytes > limit || static_cast<uint64_t>(n_win) > limit / row_bytes) {
+    char msg[200];
+    snprintf(msg, sizeof(msg),
+             "window of %lld rows x %llu channels needs more than the %llu scratch bytes of the fixed array",
+             static_cast<long long>(n_win), static_cast<unsigned long long>(hidden),
+             static_cast<unsigned long long>(limit));
     return dp::set_error(DP_ERR_CAPACITY, msg);
   }
   void* scratch = nullptr;

@@ -277,3 +277,29 @@ def test_context_refresh_checks_before_launch(m):
     assert sub(x=0) == m.ERR_INVALID_ARG
     assert c2.len[0] == 5
     assert sub(n=0) == m.OK and c2.len[0] == 0
+
+
+def test_noalloc_scratch_size_and_capacity_checks(m):
+    """The binding's NOALLOC_SCRATCH_BYTES is the header's DP_NOALLOC_SCRATCH_BYTES, and
+    dp_window_step_noalloc rejects windows beyond it (absurd sizes included, whose byte count
+    would overflow 64 bits) before it touches the GPU."""
+    text = open(HEADER).read()
+    mt = re.search(r"#define\s+DP_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert mt is not None
+    assert m.NOALLOC_SCRATCH_BYTES == int(mt.group(1)) << int(mt.group(2))
+    blk = _blocks(m, [128, 128], 128)
+    cache = m.DpKvcache()
+
+    def call(n, H, hd, dt):
+        return m._lib.dp_window_step_noalloc(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
+                                             n, ctypes.byref(blk), ctypes.byref(cache), None,
+                                             ctypes.c_void_p(FAKE + 65536), H, hd, 0, None, None, 0, dt, None)
+
+    cap = m.NOALLOC_SCRATCH_BYTES
+    assert call(cap // (2 * 2048 * 2) + 1, 16, 128, m.BF16) == m.ERR_CAPACITY      # one bf16 row too many
+    assert call(cap // (2 * 128 * 4) + 1, 2, 64, m.F32) == m.ERR_CAPACITY          # fp32 features: 4 bytes
+    assert call(2 ** 62, 1 << 30, 1 << 30, m.BF16) == m.ERR_CAPACITY               # the product overflows
+    assert call((1 << 62) + 1, 2, 64, m.BF16) == m.ERR_CAPACITY
+    assert "scratch" in m._lib.dp_last_error_detail().decode()
+    assert call(0, 2, 64, m.BF16) == m.ERR_INVALID_ARG
+    assert cache.n_advances == 0

@@ -36,9 +36,7 @@ def test_long_run_with_coordinated_noise(dp):
     pool_cpu = make_run_pool(rc)                                  # [16, 1350, D] bf16
     frames = [r // rc.frame_rows for r in rc.block_rows]          # 2 ... 2, 1
     perms = make_noise_permutations(len(frames), pool_cpu.shape[0], seed=rc.seed + 2000)
-    lists = [[2 * b, 2 * b + 1] for b in range(W)]
-    for b in range(W, len(frames)):
-        lists.append(dp.coordinated_frames(pool_cpu.shape[0], frames[b], lists[b - 1], perms[b]))
+    lists = dp.coordinated_schedule(frames, W, perms)
     sched = O.coordinated_schedule(frames, W, perms)
     assert lists == sched
     latents = [O.gather_frames(pool_cpu, f) for f in sched]

@@ -56,6 +56,50 @@ def test_noalloc_matches_window_step_on_two_calls(dp, shape):
         assert queue_b.count == queue_a.count and queue_b.evals() == queue_a.evals()
 
 
+def test_noalloc_fp32_window_matches_window_step_and_oracle_on_two_calls(dp):
+    """The fp32 path (4-byte features in the fixed array): the tiny fp32 window (2 blocks x
+    128 rows, 128-row cache, 2 x 64 heads), two calls in a row, against dp_window_step and
+    against the float64 oracle at the fp32 bar."""
+    import oracle as O
+    cfg = step_config("tiny_f32")
+    x = make_step_inputs(cfg)
+    dev = torch.device("cuda:0")
+    H, hd, D, n = cfg.n_heads, cfg.head_dim, cfg.hidden, cfg.n_win
+    blk = dp.blocks_from_table(x["table"].to(dev), x["timesteps"], cfg.block_rows)
+    q, k, v, noise = (x[key].to(dev) for key in ("q", "k", "v", "noise"))
+
+    def state():
+        cache = dp.KVCache(cfg.cache_capacity, D, torch.float32, k=x["cache_k"].to(dev).view(1, -1, D).clone(),
+                           v=x["cache_v"].to(dev).view(1, -1, D).clone(), length=cfg.cache_len)
+        queue = dp.Queue(cfg.n_blocks, max(cfg.block_rows), D, dtype=torch.float32, device=dev)
+        for _ in range(cfg.n_blocks - 1):
+            dp.queue_push(queue, noise)
+        return cache, queue
+
+    cache_a, queue_a = state()
+    cache_b, queue_b = state()
+    kv = torch.empty(2, n, D, dtype=torch.float32, device=dev)
+    out_a = torch.empty(n, D, dtype=torch.float32, device=dev)
+    out_b = torch.empty_like(out_a)
+    mod = O.lookup(x["table"], x["timesteps"])
+    ck, cv, L = x["cache_k"], x["cache_v"], cfg.cache_len
+    for call in range(2):
+        dp.window_step(q, k, v, blk, cache_a, kv, out_a, H, hd, pop=True, queue=queue_a, push_noise=noise)
+        dp.window_step_noalloc(q, k, v, blk, cache_b, out_b, H, hd, pop=True, queue=queue_b, push_noise=noise)
+        dp.device_status()
+        got = out_b.cpu().double().numpy()
+        assert_close(got, out_a.cpu().double().numpy(), "f32", f"call {call} vs dp_window_step")
+        want, kp, vp = O.window_step(x["q"], x["k"], x["v"], ck, cv, L, cfg.row_offset, mod, H, hd)
+        assert_close(got, want, "f32", f"call {call} vs the oracle")
+        n0 = cfg.block_rows[0]
+        assert cache_b.length == cache_a.length == n0
+        assert bytes_equal(cache_b.k[0, :n0], cache_a.k[0, :n0])
+        assert bytes_equal(cache_b.v[0, :n0], cache_a.v[0, :n0])
+        assert queue_b.count == queue_a.count and queue_b.evals() == queue_a.evals()
+        # the second call attends to the cache the first one wrote: the head block's k', v'
+        ck, cv, L = cache_b.k[0, :n0].cpu(), cache_b.v[0, :n0].cpu(), n0
+
+
 def test_noalloc_rejects_windows_beyond_its_scratch(dp):
     H, hd = 16, 128
     n = dp.NOALLOC_SCRATCH_BYTES // (2 * H * hd * 2) + 1   # one row too many
