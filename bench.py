@@ -3,10 +3,19 @@
 One step = the whole hot path on one window: per-block adaLN lookup (host), K/V
 modulation prepass, tensor-core window attention over [cache ; window] with the fused Q
 prologue and gate epilogue, and the queue/cache advance (head block -> cache, fresh noise
-block pushed).  Default workload: the CogVideoX-like window (4 blocks x 2700 tokens,
-2700-token cache, 48 x 64 heads, bf16).
+block pushed).  Default workload: the largest window that runs on one GPU, the shape
+sweep's 131,072-token window (4 blocks x 32,768 tokens, 32,768-token cache, 16 x 128
+heads, bf16).  The default run also times, each in its own timed region with its own clock
+record, the Wan-like window (8 x 6,240 tokens, 12 x 128 heads), the long run's steady-state
+window (8 x 2,700 tokens, 24 x 64 heads) and the whole 850-step long run, under
+"target_configs" (--no-extra skips them).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+The roofline peak is the measured dense bf16 GEMM peak that matches the timed region's
+clocks: the sustained figure (measured back to back for seconds under the power cap) when
+sw_power_cap was active during a timed region of a second or more, else the burst figure;
+both fractions are reported.
 
 N > 1 runs under torch.distributed.run, one process per GPU; every rank runs an
 independent replica (the step needs no exchange between GPUs), the timed region is
@@ -60,6 +69,36 @@ def load_peaks():
                 "source": "measured"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def choose_peak(peaks, clocks, timed_s: float):
+    """The bf16 peak that matches how the timed region ran: the sustained figure was measured
+    as a seconds-long GEMM loop under the 1 kW power cap, the burst one as short runs at full
+    clock.  The sustained one applies when sw_power_cap was active during a timed region of at
+    least a second; otherwise the burst one."""
+    reasons = (clocks or {}).get("reasons") or []
+    capped = "sw_power_cap" in reasons
+    if capped and timed_s >= 1.0:
+        kind, why = "bf16_tflops_sustained", f"sw_power_cap active over a {timed_s:.1f} s timed region"
+    else:
+        kind = "bf16_tflops"
+        why = ("no power cap in the clock record" if not capped
+               else f"sw_power_cap active but the timed region is only {timed_s:.2f} s")
+    return {"peak": peaks[kind], "kind": f"{kind} ({peaks['source']})", "why": why,
+            "burst": peaks["bf16_tflops"], "sustained": peaks["bf16_tflops_sustained"]}
+
+
+def roofline_fracs(achieved, pk):
+    if not achieved:
+        return {"frac": None, "frac_of_burst": None, "frac_of_sustained": None}
+    return {"frac": achieved / pk["peak"], "frac_of_burst": achieved / pk["burst"],
+            "frac_of_sustained": achieved / pk["sustained"]}
+
+
+DEFAULT_CONFIG = "sweep_131072"
+# timed steps when --steps is not given: about a few seconds of timed work per workload
+DEFAULT_STEPS = {"sweep_131072": 30, "wan_bf16": 80, "longrun_steady_bf16": 300}
+EXTRA_CONFIGS = ["wan_bf16", "longrun_steady_bf16", "long_run"]
 
 
 def workload(name: str):
@@ -134,7 +173,8 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def gpu_arm(args, rank: int, world: int, local_rank: int):
+def gpu_arm(args, rank: int, world: int, local_rank: int, config: str = None, steps: int = None,
+            with_e2e: bool = True):
     import torch
     import torch.distributed as dist
 
@@ -143,7 +183,9 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = workload(args.config)
+    config = config or args.config
+    steps = steps or args.steps
+    cfg = workload(config)
     if cfg.dtype != "bf16":
         raise SystemExit("bench workloads are bf16")
     x = make_step_inputs(cfg)
@@ -181,9 +223,9 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    dp.profile_begin(args.steps)
+    dp.profile_begin(steps)
     t0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
@@ -194,6 +236,9 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     dp.device_status()
     ms = t0.elapsed_time(t1)
     attn_ms, mod_ms, adv_ms = attn_ms / n_prof, mod_ms / n_prof, adv_ms / n_prof
+    if not with_e2e:
+        ms, attn_ms, mod_ms, adv_ms = max_over_ranks([ms, attn_ms, mod_ms, adv_ms], dev)
+        return cfg, dict(ms=ms, steps=steps, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms, clocks=clocks)
 
     # ---- e2e: the same step through the public API from pinned host buffers, every step's
     # inputs copied in and its output read back inside the timed region (the library's
@@ -201,7 +246,7 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
     hq, hk, hv = (x[key].pin_memory() for key in ("q", "k", "v"))
     hnoise = x["noise"].pin_memory()
     hout = torch.empty(n, D, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
+    e2e_steps = max(3, min(steps, 50))
     pipe = dp.StepPipeline(n, D, noise.shape[0], device=dev)
 
     def e2e_step():
@@ -225,12 +270,13 @@ def gpu_arm(args, rank: int, world: int, local_rank: int):
 
     # slowest rank sets the time
     ms, e2e_ms, attn_ms, mod_ms, adv_ms = max_over_ranks([ms, e2e_ms, attn_ms, mod_ms, adv_ms], dev)
-    return cfg, dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
-                     clocks=clocks,
+    return cfg, dict(ms=ms, steps=steps, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, mod_ms=mod_ms,
+                     adv_ms=adv_ms, clocks=clocks,
                      h2d=(hq.numel() + hk.numel() + hv.numel() + hnoise.numel()) * eb, d2h=hout.numel() * eb)
 
 
-def long_run_arm(args, rank: int, world: int, local_rank: int):
+def long_run_arm(args, rank: int, world: int, local_rank: int, config: str = None, steps: int = None,
+                 with_e2e: bool = True):
     """The whole long-video queue run (257 latent frames, 8-block window, 50 staggered
     timesteps per block): every schedule step is one window step of the library, with the
     window growing from 1 to 8 blocks, the head block exiting into the cache and fresh noise
@@ -249,6 +295,8 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    config = config or args.config
+    steps = steps or args.steps
     rc = run_config()
     H, hd, D, W, T = rc.n_heads, rc.head_dim, rc.hidden, rc.window_blocks, rc.n_timesteps
     noise_cpu = make_run_noise(rc)
@@ -260,17 +308,14 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     out = torch.empty(n_max, D, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    n_ctx = 4 if args.config == "long_run_ctx4" else 1
-    fresh_t = 0 if args.config == "long_run_fresh" else None
+    n_ctx = 4 if config == "long_run_ctx4" else 1
+    fresh_t = 0 if config == "long_run_fresh" else None
     frame_pool = None
-    if args.config == "long_run_coord":
+    if config == "long_run_coord":
         pool = make_run_pool(rc).to(dev)
         nf = [r // rc.frame_rows for r in rc.block_rows]
         perms = make_noise_permutations(len(nf), pool.shape[0], seed=rc.seed + 2000)
-        lists = [list(range(b * rc.frames_per_block, (b + 1) * rc.frames_per_block)) for b in range(W)]
-        for b in range(W, len(nf)):
-            lists.append(dp.coordinated_frames(pool.shape[0], nf[b], lists[b - 1], perms[b]))
-        frame_pool = (pool, lists)
+        frame_pool = (pool, dp.coordinated_schedule(nf, W, perms))
 
     def new_state():
         return (dp.KVCache(rc.slot_rows, D, torch.float16, n_slots=n_ctx, device=dev),
@@ -317,9 +362,9 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    dp.profile_begin(args.steps)
+    dp.profile_begin(steps)
     t0.record(stream)
-    n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=args.steps,
+    n_steps = dp.run_fifo(noise, table, tau, W, cache, queue, kv, out, H, hd, on_step=on_step, max_steps=steps,
                           cache_all_slots=n_ctx > 1, frame_pool=frame_pool, fresh_t=fresh_t)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -342,6 +387,13 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     dp.device_status()
     ms = t0.elapsed_time(t1)
+    tokens = sum(steps_n)
+    flop = sum(4 * n * (lc + n) * hd * H for n, lc in zip(steps_n, steps_lc))
+    if not with_e2e:
+        ms, attn_ms = max_over_ranks([ms, attn_ms], dev)
+        return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
+                    clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx, fresh=fresh_t is not None,
+                    steady=steady)
 
     # e2e: the same run through the public API with every pushed noise block copied from
     # pinned host memory right before its push and every step's output read back to the host
@@ -399,7 +451,7 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     if e2e_pool is not None:
         e2e_pool[0].copy_(hpool, non_blocking=True)
     n_e2e = dp.run_fifo(hb, table, tau, W, cache, queue, kv, outs, H, hd, on_step=on_step_e2e,
-                        max_steps=args.steps, cache_all_slots=n_ctx > 1, frame_pool=e2e_pool, fresh_t=fresh_t)
+                        max_steps=steps, cache_all_slots=n_ctx > 1, frame_pool=e2e_pool, fresh_t=fresh_t)
     for ev in read_done:
         if ev is not None:
             stream.wait_event(ev)
@@ -407,25 +459,24 @@ def long_run_arm(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     dp.device_status()
-    tokens = sum(steps_n)
-    flop = sum(4 * n * (lc + n) * hd * H for n, lc in zip(steps_n, steps_lc))
     ms, e2e_ms, attn_ms = max_over_ranks([ms, e2e_ms, attn_ms], dev)
     return dict(ms=ms, steps=n_steps, tokens=tokens, flop=flop, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms,
                 e2e_ms=e2e_ms, e2e_steps=n_e2e, h2d=hb.h2d / max(n_e2e, 1), d2h=d2h[0] / max(n_e2e, 1),
                 clocks=clocks, rc=rc, launches=launches[0], n_ctx=n_ctx, fresh=fresh_t is not None, steady=steady)
 
 
-def long_run_line(args, world, r):
+def long_run_line(args, world, r, config: str = None):
     peaks = load_peaks()
+    config = config or args.config
     rc = r["rc"]
     achieved = r["flop"] / (r["attn_ms"] / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    pk = choose_peak(peaks, r["clocks"], r["ms"] / 1e3)
     steady_flop = 4 * 21600 * (21600 + r["n_ctx"] * 2700) * rc.head_dim * rc.n_heads
     return {
         "metric": METRIC, "value": world * r["tokens"] / (r["ms"] / 1e3), "unit": "tokens/s", "n_gpus": world,
         "steps": r["steps"], "warmup": args.warmup, "ms_per_step": r["ms"] / r["steps"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": (f"{args.config}: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
+        "config": {"workload": (f"{config}: {rc.n_frames} latent frames x {rc.frame_rows} tokens in "
                                 f"{rc.frames_per_block}-frame blocks, window of {rc.window_blocks} blocks, "
                                 f"{rc.n_timesteps} staggered timesteps per block, {rc.n_heads}x{rc.head_dim} heads, "
                                 f"bf16, cache of the last {r['n_ctx']} exited block(s)"
@@ -439,16 +490,15 @@ def long_run_line(args, world, r):
         "stage_ms": {"modulate": r["mod_ms"] / r["steps"], "attention": r["attn_ms"] / r["steps"],
                      "advance": r["adv_ms"] / r["steps"],
                      "outside_stages": (r["ms"] - r["mod_ms"] - r["attn_ms"] - r["adv_ms"]) / r["steps"]},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["peak"], "unit": "TFLOP/s",
+                     **roofline_fracs(achieved, pk), "traffic": None,
                      "traffic_unit": "bytes per launch (not captured for the run: window sizes vary per step)",
-                     "kernel": "window_attn_tc_kernel",
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "kernel": "window_attn_tc_kernel", "peak_kind": pk["kind"], "peak_why": pk["why"],
                      "algorithmic_flop_per_run": r["flop"], "steady_state_flop_per_launch": steady_flop},
         "clocks": r["clocks"],
-        "e2e": {"value": world * r["tokens"] / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": None,
+        "e2e": ({"value": world * r["tokens"] / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]} if "e2e_ms" in r else None),
+        "gpu_launches": r["launches"],
     }
 
 
@@ -577,11 +627,12 @@ def sublayer_line(args, world, cfg, r):
     attn_flop = cfg.attn_flop()
     qkv_flop = 2 * n * D * 3 * D
     out_flop = 2 * n * D * D
-    peak = peaks["bf16_tflops_sustained"]
+    pk = choose_peak(peaks, r["clocks"], r["ms"] / 1e3)
+    peak = pk["peak"]
     tf = lambda flop, ms: flop / (ms / 1e3) / 1e12 if ms > 0 else None
     achieved = tf(attn_flop, attn_ms)
     ln_bytes = 2 * n * D * 2
-    adv_bytes = (4 * cfg.block_rows[0] + 3 * cfg.push_rows) * D * 2
+    adv_bytes = (4 * cfg.block_rows[0] + 2 * cfg.push_rows) * D * 2
     gbs = lambda b, ms: b / (ms / 1e3) / 1e9 if ms > 0 else None
     ms_step = r["ms"] / args.steps
     n_ctx = r["n_ctx"]
@@ -601,9 +652,9 @@ def sublayer_line(args, world, cfg, r):
         "stage_ms": {"ln_modulate": ln_ms, "qkv_projection": qkv_ms, "attention": attn_ms,
                      "out_projection": out_ms, "advance": adv_ms},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     **roofline_fracs(achieved, pk), "traffic": None,
                      "traffic_unit": "bytes per launch (see the window-step configurations)",
-                     "kernel": "window_attn_tc_kernel", "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "kernel": "window_attn_tc_kernel", "peak_kind": pk["kind"], "peak_why": pk["why"],
                      "algorithmic_flop_per_launch": attn_flop},
         "stage_tensor": {
             "qkv_projection": {"flop": qkv_flop, "ms": qkv_ms, "achieved_tflops": tf(qkv_flop, qkv_ms),
@@ -614,7 +665,10 @@ def sublayer_line(args, world, cfg, r):
             "ln_modulate": {"bytes": ln_bytes, "ms": ln_ms, "achieved_gbs": gbs(ln_bytes, ln_ms),
                             "frac": (gbs(ln_bytes, ln_ms) or 0) / peaks["hbm_gbs"]},
             "advance": {"bytes": adv_bytes, "ms": adv_ms, "achieved_gbs": gbs(adv_bytes, adv_ms),
-                        "frac": (gbs(adv_bytes, adv_ms) or 0) / peaks["hbm_gbs"]}},
+                        "frac": (gbs(adv_bytes, adv_ms) or 0) / peaks["hbm_gbs"],
+                        "mirror_write_bytes": cfg.push_rows * D * 2,
+                        "note": "bytes = 4 n_exit D e + 2 n_push D e (algorithmic); the push's second write into "
+                                "the mirrored latent ring (mirror_write_bytes) is overhead, not counted"}},
         "clocks": r["clocks"],
         "e2e": {"value": world * n / (r["e2e_ms"] / r["e2e_steps"] / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
@@ -700,16 +754,18 @@ def sublayer_cpu_baseline(cfg, budget_s: float = 12.0, fresh: bool = False):
 def stage_hbm(cfg, r, peaks):
     """Achieved HBM bandwidth of the two copy-like stages (algorithmic bytes / event time):
     modulation reads k, v and writes k', v' (4 N_w D e bytes); the advance copies the head
-    block's k'/v' into the cache (4 n_exit D e) and the noise block into both halves of the
-    mirrored ring (3 n_push D e)."""
+    block's k'/v' into the cache (4 n_exit D e) and pushes the noise block (read and write,
+    2 n_push D e).  The push also writes the block a second time, into the mirror half of the
+    latent ring (n_push D e): overhead of the layout, reported apart and not counted."""
     eb = cfg.elem_bytes
     mod_b = 4 * cfg.n_win * cfg.hidden * eb
-    adv_b = (4 * cfg.block_rows[0] + 3 * cfg.push_rows) * cfg.hidden * eb
+    adv_b = (4 * cfg.block_rows[0] + 2 * cfg.push_rows) * cfg.hidden * eb
     out = {}
     for name, b, ms in (("modulate", mod_b, r["mod_ms"]), ("advance", adv_b, r["adv_ms"])):
         gbs = b / (ms / 1e3) / 1e9 if ms > 0 else None
         out[name] = {"bytes": b, "ms": ms, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
                      "frac": (gbs / peaks["hbm_gbs"]) if gbs else None}
+    out["advance"]["mirror_write_bytes"] = cfg.push_rows * cfg.hidden * eb
     return out
 
 
@@ -835,17 +891,87 @@ def reference_arm(args):
 
 # ----------------------------------------------------------------------------- main
 
+def step_line(args, world, cfg, r, config: str):
+    """The JSON record of a window-step workload (the main line, or one of target_configs)."""
+    peaks = load_peaks()
+    flop = cfg.attn_flop()
+    steps = r["steps"]
+    achieved = flop / (r["attn_ms"] / 1e3) / 1e12
+    pk = choose_peak(peaks, r["clocks"], r["ms"] / 1e3)
+    line = {
+        "metric": METRIC, "value": job_throughput(world, cfg.n_win, steps, r["ms"]), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": r["ms"] / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(cfg), "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": f"inputs larger than L2 (q, k, v {3 * cfg.n_win * cfg.hidden * 2 / 2**20:.0f} MiB "
+                         f"> {L2_BYTES / 2**20:.0f} MiB)"},
+        "attn_tflops": achieved,
+        "stage_ms": {"modulate": r["mod_ms"], "attention": r["attn_ms"], "advance": r["adv_ms"]},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["peak"], "unit": "TFLOP/s",
+                     **roofline_fracs(achieved, pk), "traffic": attention_traffic(config),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                     "kernel": "window_attn_tc_kernel", "peak_kind": pk["kind"], "peak_why": pk["why"],
+                     "algorithmic_flop_per_launch": flop},
+        "stage_hbm": stage_hbm(cfg, r, peaks),
+        "clocks": r["clocks"],
+        "gpu_launches": 3 * steps,
+    }
+    if "e2e_ms" in r:
+        line["e2e"] = {"value": world * cfg.n_win / (r["e2e_ms"] / r["e2e_steps"] / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]}
+    return line
+
+
+def compact(line):
+    """The figures of a target_configs entry."""
+    rf = line["roofline"]
+    out = {"workload": line["config"]["workload"], "value": line["value"], "unit": line["unit"],
+           "steps": line["steps"], "ms_per_step": line["ms_per_step"], "attn_tflops": line["attn_tflops"],
+           "attention_ms_per_step": line["stage_ms"]["attention"],
+           "roofline": {k: rf[k] for k in ("achieved", "peak", "frac", "frac_of_burst", "frac_of_sustained",
+                                           "peak_kind", "peak_why", "traffic") if k in rf},
+           "clocks": line["clocks"]}
+    if "full_window_step_ms" in line:
+        out["full_window_step_ms"] = line["full_window_step_ms"]
+    if "stage_hbm" in line:
+        out["stage_hbm"] = {k: {"achieved_gbs": v["achieved_gbs"], "frac": v["frac"]}
+                            for k, v in line["stage_hbm"].items()}
+    return out
+
+
+def extra_lines(args, rank: int, world: int, local_rank: int):
+    """The other target workloads, each timed in its own region: the Wan-like window, the long
+    run's steady-state window and the whole long run (no e2e or CPU baseline for these)."""
+    out = {}
+    for name in EXTRA_CONFIGS:
+        if name == "long_run":
+            r = long_run_arm(args, rank, world, local_rank, config=name, steps=850, with_e2e=False)
+            if rank == 0:
+                out[name] = compact(long_run_line(args, world, r, config=name))
+        else:
+            cfg, r = gpu_arm(args, rank, world, local_rank, config=name, steps=DEFAULT_STEPS[name], with_e2e=False)
+            if rank == 0:
+                out[name] = compact(step_line(args, world, cfg, r, name))
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="cogvideo_bf16")
+    ap.add_argument("--config", default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the target_configs timings of the default run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    default_run = args.config is None
+    if args.config is None:
+        args.config = DEFAULT_CONFIG
+    if args.steps is None:
+        args.steps = 850 if args.config.startswith("long_run") else DEFAULT_STEPS.get(args.config, 300)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -865,66 +991,30 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     if args.config in ("long_run", "long_run_ctx4", "long_run_coord", "long_run_fresh"):
-        if args.steps == 300 and "--steps" not in sys.argv:
-            args.steps = 850                 # the whole run
         r = long_run_arm(args, rank, world, local_rank)
         if rank == 0:
             line = long_run_line(args, world, r)
-            line["gpu_launches"] = r["launches"] if "launches" in r else None
             if not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(workload("long_run"))
                 line["cpu_baseline"]["sample"] = "steady-state step of the run: " + line["cpu_baseline"]["sample"]
             print(json.dumps(line), flush=True)
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-    if args.config.startswith("sublayer_"):
+    elif args.config.startswith("sublayer_"):
         cfg, r = sublayer_arm(args, rank, world, local_rank)
         if rank == 0:
             line = sublayer_line(args, world, cfg, r)
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = sublayer_cpu_baseline(cfg, fresh=args.config.startswith("sublayer_fresh_"))
             print(json.dumps(line), flush=True)
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-    cfg, r = gpu_arm(args, rank, world, local_rank)
-    if rank == 0:
-        peaks = load_peaks()
-        flop = cfg.attn_flop()
-        ms_step = r["ms"] / args.steps
-        value = job_throughput(world, cfg.n_win, args.steps, r["ms"])
-        achieved = flop / (r["attn_ms"] / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        e2e_ms_step = r["e2e_ms"] / r["e2e_steps"]
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": describe(cfg), "parallelism": f"replicas x{world} (no exchange)",
-                       "l2": f"inputs larger than L2 (q, k, v {3 * cfg.n_win * cfg.hidden * 2 / 2**20:.0f} MiB "
-                             f"> {L2_BYTES / 2**20:.0f} MiB)"},
-            "attn_tflops": achieved,
-            "stage_ms": {"modulate": r["mod_ms"], "attention": r["attn_ms"], "advance": r["adv_ms"]},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": attention_traffic(args.config),
-                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                         "kernel": "window_attn_tc_kernel",
-                         "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
-                         "algorithmic_flop_per_launch": flop},
-            "stage_hbm": stage_hbm(cfg, r, peaks),
-            "clocks": r["clocks"],
-            "e2e": {"value": world * cfg.n_win / (e2e_ms_step / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-            "gpu_launches": 3 * args.steps,
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg)
-        print(json.dumps(line), flush=True)
+    else:
+        cfg, r = gpu_arm(args, rank, world, local_rank)
+        line = step_line(args, world, cfg, r, args.config) if rank == 0 else None
+        extras = extra_lines(args, rank, world, local_rank) if default_run and not args.no_extra else None
+        if rank == 0:
+            if extras:
+                line["target_configs"] = extras
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(cfg)
+            print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
