@@ -97,6 +97,66 @@ def test_attention_bf16_matches_oracle(dp, case):
     assert_close(out.cpu().double().numpy(), want, "bf16", f"attention {case}")
 
 
+def _jump_case(hd, cache_len, n_win, seed=31):
+    """Queries in groups of 128 rows, each group with its own direction (dim g of every head);
+    keys planted on that direction at chosen logit levels (log2 units: x = q.k * scale *
+    log2(e)), so that the running reference max of the softmax jumps by more than 2^8 in
+    chosen 32-key chunks of chosen key tiles, with groups of keys just below each jump
+    carrying a visible share of the row's weight.  Key index = position in [cache ; window]."""
+    BN = 128 if hd == 64 else 64
+    nch = BN // 32
+    key = lambda t, i, o: t * BN + 32 * min(i, nch - 1) + o
+    plan = {   # every group on tiles of its own
+        0: [(key(1, c, o), 3.0) for c in range(nch - 1) for o in range(32)] + [(key(1, nch - 1, 5), 11.5)],
+        1: [(key(2, 0, o), 3.0) for o in range(31) if o != 7] + [(key(2, 0, 7), 11.6)],
+        2: [(key(3, 1, 3), 9.0), (key(6, nch - 2, 10), 18.0)],
+        3: [(key(4, 0, o), 2.0) for o in range(1, 32)] + [(key(4, 0, 0), 9.0), (key(4, nch - 1, 31), 18.2)],
+    }
+    assert len({j for keys in plan.values() for j, _ in keys}) == sum(len(keys) for keys in plan.values())
+    H = 2
+    D = H * hd
+    g = torch.Generator().manual_seed(seed)
+    L = cache_len + n_win
+    q = torch.randn(n_win, D, generator=g) * 0.5
+    kall = torch.randn(L, D, generator=g) * 0.05
+    vall = torch.randn(L, D, generator=g)
+    a, s = 4.0, hd ** -0.5
+    for h in range(H):
+        q[:, h * hd:h * hd + 4] = 0.0
+        for grp, keys in plan.items():
+            rows = slice(128 * grp, 128 * (grp + 1))
+            q[rows, h * hd + grp] = a
+            for j, x in keys:
+                kall[j, h * hd:h * hd + 4] = 0.0
+                kall[j, h * hd + grp] = x / (a * s * 1.4426950408889634)
+    q = q.to(torch.bfloat16)
+    kall, vall = kall.to(torch.float16), vall.to(torch.float16)
+    return H, D, q, kall[cache_len:].contiguous(), vall[cache_len:].contiguous(), kall[:cache_len].contiguous(), \
+        vall[:cache_len].contiguous()
+
+
+@pytest.mark.parametrize("hd,cache_len", [(64, 0), (64, 168), (128, 0), (128, 100)])
+def test_attention_reference_max_jumps_mid_tile(dp, hd, cache_len):
+    """The softmax's reference max moves by more than 2^8 inside a key tile (in its first,
+    middle and last 32-key chunk, twice in one tile, over a ragged cache-window boundary):
+    O, the row sum and the P chunks already computed are rescaled."""
+    n = 1024
+    H, D, q, k, v, ck, cv = _jump_case(hd, cache_len, n)
+    cap = max(cache_len, 1)
+    ckd = ck.cuda() if cache_len else torch.zeros(cap, D, dtype=torch.float16, device="cuda")
+    cvd = cv.cuda() if cache_len else torch.zeros(cap, D, dtype=torch.float16, device="cuda")
+    table = _table(D)
+    blk = dp.blocks_from_table(table.cuda(), [0], [n])
+    out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
+    dp.window_attention(q.cuda(), k.cuda(), v.cuda(), ckd, cvd, cache_len, out, H, hd, blk, flags=0)
+    dp.device_status()
+    want = O.window_attention(q, k, v, ck if cache_len else ckd.cpu(), cv if cache_len else cvd.cpu(), cache_len,
+                              blk.offsets, O.lookup(table, [0]), H, hd, mod_q=False, gate_out=False)
+    assert_close(out.cpu().double().numpy(), want, "bf16", f"max jumps hd {hd} cache {cache_len}")
+    # the planted keys decide the result: each group's output is far from the mean of V
+    assert np.abs(want[:512]).max() > 0.5
+
+
 def test_attention_bf16_deterministic(dp):
     H, hd, n, Lc = 4, 64, 1000, 300
     D = H * hd
