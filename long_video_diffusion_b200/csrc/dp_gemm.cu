@@ -23,9 +23,14 @@
 //              whose residual loads run one chunk ahead); it frees the accumulator for the
 //              tile after next, so a tile's epilogue runs while the next tile's products
 //              accumulate
-// Tiles are numbered in groups of kGroupM m tiles: within a group the m tiles of one n tile
-// are consecutive, so the ~148 tiles in flight span about 16 row blocks of A and 9 column
-// blocks of W (about 27 MB at hidden 3072) instead of whole rows of W.
+// Tiles are numbered in groups of group_m m tiles: within a group the m tiles of one n tile
+// are consecutive, so the ~148 tiles in flight span the group's row blocks of A and a few
+// column blocks of W.  A group's rows of A stay in L2 while the group sweeps all of W.  A W
+// that fits in L2 with room to spare (up to kSmallWBytes) stays there across groups, and
+// groups of 16 row blocks keep the rows of A (and of the residual) in flight small; a larger
+// W is read from DRAM once per group, so the host then makes the groups as large as about
+// kGroupABytes of A allows (equal in size), which reads W a couple of times instead of once
+// per 16 row blocks.
 // Every wait is bounded (dp_device.cuh): on giving up the kernel records a timeout in the
 // device status word, stops, drains its own copies and products, frees TMEM and returns.
 #include <atomic>
@@ -42,14 +47,17 @@ namespace {
 
 constexpr int GBM = 128;  // output rows per tile
 constexpr int GBK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGroupM = 16;  // m tiles per group of the tile order
+constexpr int kGroupMSmall = 16;               // m tiles per group while W stays in L2
+constexpr int64_t kSmallWBytes = 24ll << 20;   // W up to this size stays in L2 across groups
+constexpr int64_t kGroupABytes = 34ll << 20;   // rows of A a group covers when W does not
 
 // Tile t of the grouped order -> (m tile, n tile).
-__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles_n, int& m_tile, int& n_tile) {
-  const int per_group = kGroupM * n_tiles_n;
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles_n, int group_m, int& m_tile,
+                                            int& n_tile) {
+  const int per_group = group_m * n_tiles_n;
   const int group = t / per_group;
-  const int first_m = group * kGroupM;
-  const int gm = min(kGroupM, m_tiles - first_m);
+  const int first_m = group * group_m;
+  const int gm = min(group_m, m_tiles - first_m);
   const int within = t - group * per_group;
   m_tile = first_m + within % gm;
   n_tile = within / gm;
@@ -79,6 +87,7 @@ struct GemmParams {
   int32_t n;
   int32_t k;
   int32_t n_tiles_n;
+  int32_t group_m;  // m tiles per group of the tile order
   int32_t m_tiles;
   int32_t n_tiles;
   const float* bias;               // [n] or NULL
@@ -212,7 +221,7 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       bool ok = true;
       for (int i = 0; ok && i < n_mine; ++i) {
         int m_tile, n_tile;
-        tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, m_tile, n_tile);
+        tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, p.group_m, m_tile, n_tile);
         for (int kt = 0; kt < KT; ++kt) {
           const int g = issued;
           const int s = g % L::STAGES;
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(GemmLayout<BN>::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       int m_tile, n_tile;
-      tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, m_tile, n_tile);
+      tile_coords(blockIdx.x + i * gridDim.x, p.m_tiles, p.n_tiles_n, p.group_m, m_tile, n_tile);
       const int64_t row = static_cast<int64_t>(m_tile) * GBM + quarter * 32 + lane;
       const uint32_t taddr = tmem + tlane + static_cast<uint32_t>(b * BN);
       const bool row_ok = row < p.m;
@@ -343,6 +352,15 @@ cudaError_t launch_bn(const GemmArgs& g, cudaStream_t s) {
   if (n_tiles > 0x7fffffff) return cudaErrorInvalidValue;
   p.m_tiles = static_cast<int32_t>(m_tiles);
   p.n_tiles = static_cast<int32_t>(n_tiles);
+  if (static_cast<int64_t>(g.n) * g.k * 2 <= kSmallWBytes) {
+    p.group_m = kGroupMSmall;
+  } else {
+    // as few groups as keep a group's rows of A within kGroupABytes, all of about one size
+    const int64_t a_tile_bytes = static_cast<int64_t>(GBM) * g.k * 2;
+    int64_t groups = (m_tiles * a_tile_bytes + kGroupABytes - 1) / kGroupABytes;
+    groups = groups < 1 ? 1 : (groups > m_tiles ? m_tiles : groups);
+    p.group_m = static_cast<int32_t>((m_tiles + groups - 1) / groups);
+  }
   p.bias = g.bias;
   p.y0 = g.y0;
   p.y1 = g.y1;
