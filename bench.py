@@ -43,7 +43,8 @@ METRIC = "window-step tokens/s and attention TFLOP/s (fraction of bf16 peak) at 
 # profiles/), valid only for the kernel source they were captured on (md5 over
 # csrc/dp_attn_tc.cu and csrc/dp_device.cuh); any other source reports null.
 TRAFFIC_SOURCE_MD5 = "0f4d0a643530e059790321993f0188af"
-TRAFFIC_BYTES = {"cogvideo_bf16": 233.596416e6 + 50.829312e6, "wan_bf16": 633.475072e6 + 142.530048e6}
+TRAFFIC_BYTES = {"cogvideo_bf16": 233.596416e6 + 50.829312e6, "wan_bf16": 633.475072e6 + 142.530048e6,
+                 "sweep_16384": 236.308736e6 + 51.109632e6, "sweep_131072": 9532.882944e6 + 564.817408e6}
 L2_BYTES = 126 * 1024 * 1024
 
 
