@@ -241,6 +241,26 @@ def gpu_arm(args, rank: int, world: int, local_rank: int, config: str = None, st
         ms, attn_ms, mod_ms, adv_ms = max_over_ranks([ms, attn_ms, mod_ms, adv_ms], dev)
         return cfg, dict(ms=ms, steps=steps, attn_ms=attn_ms, mod_ms=mod_ms, adv_ms=adv_ms, clocks=clocks)
 
+    # ---- the two HBM-bound kernels timed alone, back to back on the same bytes (the stage
+    # events above hold each launch's gap and run at the SM clock the attention leaves behind,
+    # power-capped on the large workloads)
+    def t_alone(fn, iters=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(iters):
+            fn()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        return a0.elapsed_time(a1) / iters
+
+    n0 = cfg.block_rows[0]
+    mod_alone_ms = t_alone(lambda: (dp.adaln_modulate(k, kv[0], blk), dp.adaln_modulate(v, kv[1], blk)))
+    adv_alone_ms = t_alone(lambda: dp.kvcache_advance(cache, kv[0][:n0], kv[1][:n0], n0))
+    dp.device_status()
+
     # ---- e2e: the same step through the public API from pinned host buffers, every step's
     # inputs copied in and its output read back inside the timed region (the library's
     # StepPipeline overlaps step i's copies with step i - 1's compute on three streams)
@@ -270,9 +290,10 @@ def gpu_arm(args, rank: int, world: int, local_rank: int, config: str = None, st
     dp.device_status()
 
     # slowest rank sets the time
-    ms, e2e_ms, attn_ms, mod_ms, adv_ms = max_over_ranks([ms, e2e_ms, attn_ms, mod_ms, adv_ms], dev)
+    ms, e2e_ms, attn_ms, mod_ms, adv_ms, mod_alone_ms, adv_alone_ms = max_over_ranks(
+        [ms, e2e_ms, attn_ms, mod_ms, adv_ms, mod_alone_ms, adv_alone_ms], dev)
     return cfg, dict(ms=ms, steps=steps, e2e_ms=e2e_ms, e2e_steps=e2e_steps, attn_ms=attn_ms, mod_ms=mod_ms,
-                     adv_ms=adv_ms, clocks=clocks,
+                     adv_ms=adv_ms, mod_alone_ms=mod_alone_ms, adv_alone_ms=adv_alone_ms, clocks=clocks,
                      h2d=(hq.numel() + hk.numel() + hv.numel() + hnoise.numel()) * eb, d2h=hout.numel() * eb)
 
 
@@ -767,6 +788,14 @@ def stage_hbm(cfg, r, peaks):
         out[name] = {"bytes": b, "ms": ms, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
                      "frac": (gbs / peaks["hbm_gbs"]) if gbs else None}
     out["advance"]["mirror_write_bytes"] = cfg.push_rows * cfg.hidden * eb
+    # the same kernels alone (no launch gap, no power-capped clock inherited from the attention):
+    # the prepass over k and v, and the advance's cache write (the head block's k', v')
+    for name, b, key in (("modulate_alone", mod_b, "mod_alone_ms"),
+                         ("advance_cache_alone", 4 * cfg.block_rows[0] * cfg.hidden * eb, "adv_alone_ms")):
+        if key in r and r[key] > 0:
+            gbs = b / (r[key] / 1e3) / 1e9
+            out[name] = {"bytes": b, "ms": r[key], "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+                         "frac": gbs / peaks["hbm_gbs"]}
     return out
 
 
