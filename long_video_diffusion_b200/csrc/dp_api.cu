@@ -1055,11 +1055,15 @@ dp_status dp_fifo_plan(const dp_fifo* f, const dp_queue* q, dp_fifo_step* out) {
     *out = o;
     return DP_OK;
   }
-  // live blocks at step s: [lo, hi), e_b <= s < e_b + T
-  int64_t lo = 0;
-  while (lo < f->n_blocks && entry_step(lo, T, W) + T <= s) ++lo;
-  int64_t hi = lo;
-  while (hi < f->n_blocks && entry_step(hi, T, W) <= s) ++hi;
+  // live blocks at step s: [lo, hi), e_b <= s < e_b + T.  floor(b T / W) >= x holds exactly
+  // for b >= ceil(x W / T) (x > 0), so lo and hi are the first blocks with e_b >= s - T + 1
+  // and with e_b >= s + 1.
+  auto first_entering_at_or_after = [&](int64_t x) -> int64_t {
+    const int64_t b = x <= 0 ? 0 : (x * W + T - 1) / T;
+    return b < f->n_blocks ? b : f->n_blocks;
+  };
+  const int64_t lo = first_entering_at_or_after(s - T + 1);
+  const int64_t hi = first_entering_at_or_after(s + 1);
   if (hi != f->next_block || q->count != hi - lo)
     return fail(DP_ERR_INVALID_ARG, "queue does not match the schedule at step %lld: %d live blocks, %lld expected "
                 "(blocks %lld..%lld entered, next %d)", static_cast<long long>(s), q->count,
