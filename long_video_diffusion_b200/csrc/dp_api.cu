@@ -984,7 +984,9 @@ dp_status dp_sublayer_step(const void* x, int64_t n_win, const dp_blocks* blk, c
 
 namespace {
 
-// floor(b * T / W): entry step of block b (the review's Figure 1 stagger, made exact).
+// floor(b * T / W): the entry step of block b.  The pages show blocks entering one after
+// another without giving the stagger; this one keeps W blocks live in the steady state and
+// gives every block T evaluations.
 int64_t entry_step(int64_t b, int32_t T, int32_t W) { return b * T / W; }
 
 dp_status check_fifo(const dp_fifo* f) {
