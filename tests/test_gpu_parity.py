@@ -97,7 +97,7 @@ def test_attention_bf16_matches_oracle(dp, case):
     assert_close(out.cpu().double().numpy(), want, "bf16", f"attention {case}")
 
 
-def _jump_case(hd, cache_len, n_win, seed=31):
+def _jump_case(hd, cache_len, n_win, seed=31, levels=None):
     """Queries in groups of 128 rows, each group with its own direction (dim g of every head);
     keys planted on that direction at chosen logit levels (log2 units: x = q.k * scale *
     log2(e)), so that the running reference max of the softmax jumps by more than 2^8 in
@@ -106,7 +106,7 @@ def _jump_case(hd, cache_len, n_win, seed=31):
     BN = 128 if hd == 64 else 64
     nch = BN // 32
     key = lambda t, i, o: t * BN + 32 * min(i, nch - 1) + o
-    plan = {   # every group on tiles of its own
+    plan = levels(key, nch) if levels else {   # every group on tiles of its own
         0: [(key(1, c, o), 3.0) for c in range(nch - 1) for o in range(32)] + [(key(1, nch - 1, 5), 11.5)],
         1: [(key(2, 0, o), 3.0) for o in range(31) if o != 7] + [(key(2, 0, 7), 11.6)],
         2: [(key(3, 1, 3), 9.0), (key(6, nch - 2, 10), 18.0)],
@@ -154,6 +154,41 @@ def test_attention_reference_max_jumps_mid_tile(dp, hd, cache_len):
                               blk.offsets, O.lookup(table, [0]), H, hd, mod_q=False, gate_out=False)
     assert_close(out.cpu().double().numpy(), want, "bf16", f"max jumps hd {hd} cache {cache_len}")
     # the planted keys decide the result: each group's output is far from the mean of V
+    assert np.abs(want[:512]).max() > 0.5
+
+
+# Jumps past the range of fp32 exp2 (2^x is infinite from x = 128 on): single keys 60 to 400
+# log2 units above everything before them, in columns of either exp2 unit (column 0 of a
+# 32-key chunk and its last column; column 7), some in the same tile as a smaller jump.
+def _far_levels(key, nch):
+    return {
+        0: [(key(1, 0, 0), 150.0)],
+        1: [(key(2, 0, o), 3.0) for o in range(8, 31)] + [(key(2, 0, 7), 200.0)],
+        2: [(key(3, nch - 1, 3), 60.0), (key(6, 0, 10), 300.0)],
+        3: [(key(4, 0, 0), 130.0), (key(4, nch - 1, 31), 400.0)],
+    }
+
+
+@pytest.mark.parametrize("hd,cache_len", [(64, 0), (64, 168), (128, 0), (128, 100)])
+def test_attention_reference_max_jumps_past_fp32_exp2_range(dp, hd, cache_len):
+    """Scores that jump by 60 to 400 log2 units within the row: each row's output is, to
+    within the tolerance, the value row of its largest key, whatever came before it."""
+    n = 1024
+    H, D, q, k, v, ck, cv = _jump_case(hd, cache_len, n, seed=37, levels=_far_levels)
+    cap = max(cache_len, 1)
+    ckd = ck.cuda() if cache_len else torch.zeros(cap, D, dtype=torch.float16, device="cuda")
+    cvd = cv.cuda() if cache_len else torch.zeros(cap, D, dtype=torch.float16, device="cuda")
+    table = _table(D)
+    blk = dp.blocks_from_table(table.cuda(), [0], [n])
+    out = torch.empty(n, D, dtype=torch.bfloat16, device="cuda")
+    dp.window_attention(q.cuda(), k.cuda(), v.cuda(), ckd, cvd, cache_len, out, H, hd, blk, flags=0)
+    dp.device_status()
+    want = O.window_attention(q, k, v, ck if cache_len else ckd.cpu(), cv if cache_len else cvd.cpu(), cache_len,
+                              blk.offsets, O.lookup(table, [0]), H, hd, mod_q=False, gate_out=False)
+    got = out.cpu().double().numpy()
+    assert np.isfinite(got).all()
+    assert_close(got, want, "bf16", f"far jumps hd {hd} cache {cache_len}")
+    # one key holds all the weight: the first 512 rows equal a value row of V
     assert np.abs(want[:512]).max() > 0.5
 
 
